@@ -1,0 +1,213 @@
+/*
+ * h3.h -- C ABI of libh3: packed multimodal MM-RoPE attention on B200 (sm_100a).
+ *
+ * The library computes the attention hot path of a single-stream audio-video
+ * diffusion transformer: text, reference, video-latent and stereo-audio rows
+ * are packed into ONE sequence, every row carries a three-axis (t, h, w)
+ * position, Q and K are rotated by a three-axis rotary embedding, and every
+ * row attends to every row.
+ *
+ * Sources (page titles as published):
+ *   [P1] "Inside MiniMax H3: One DiT Stream for Text, Video, and Stereo Audio",
+ *        section 2 (one packed sequence, shared projections), section 4
+ *        (three-axis RoPE on a shared physical timeline; row order carries no
+ *        position), section 6 (full attention dominates the cost).
+ *   [P3] "MiniMax H3 -- one transformer that denoises video and audio
+ *        together": latent-frame passage (880 tokens of one latent frame share
+ *        t), clock-unit passage (1 unit = 1/40 s, 5/3 units per 24 fps frame),
+ *        text passage (text t = index), rope-config passage (inverse
+ *        frequencies computed from rope_theta / rope_freq_dim), and the
+ *        bidirectional-attention passage.
+ *   [P5] "MiniMax H3 -- Open-Weights Omni-Reference Video-Audio Generation
+ *        Model Card", section H3-Omni-Transformer (3-D MM-RoPE over (t,h,w)).
+ *
+ * Conventions for every call:
+ *   - Pointers named d_* are DEVICE pointers owned by the caller; the library
+ *     never frees or retains them after the call returns.  Host pointers are
+ *     read during the call only.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream).  Arguments are validated on the host
+ *     before anything is launched; a call that returns an error launched
+ *     nothing, except H3_ERR_CUDA reported by the launch itself.
+ *   - The library allocates no device memory.  Kernel-side faults in the
+ *     inputs (a permutation entry out of range, a bounded wait that expired)
+ *     are recorded in a per-device error word; h3_check_device_error reads
+ *     and clears it.
+ *   - Q/K/V/O tensors are bf16 in row-major [batch][n_rows][n_heads][head_dim]
+ *     with a row stride of `row_stride` elements (>= n_heads * head_dim,
+ *     a multiple of 8) and a batch stride of n_rows * row_stride elements.
+ *     Base pointers must be 16-byte aligned.  This is the natural layout of a
+ *     fused QKV projection output (hidden 5376 = 42 heads x 128).
+ */
+#ifndef H3_H_
+#define H3_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  H3_OK = 0,
+  H3_ERR_INVALID_ARG = 1,   /* bad size, count, table or pointer */
+  H3_ERR_UNSUPPORTED = 2,   /* valid but not implemented (head_dim != 128, misalignment, ...) */
+  H3_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
+  H3_ERR_TIMEOUT = 4,       /* a bounded device-side wait expired (see h3_set_wait_limit_ns) */
+  H3_ERR_DEVICE_INPUT = 5   /* a kernel found a bad input (e.g. perm entry out of range) */
+} h3_status;
+
+/* Segment kinds. */
+enum { H3_SEG_TEXT = 0, H3_SEG_VIDEO = 1, H3_SEG_AUDIO = 2 };
+
+/* Segment flags (bit set). */
+enum {
+  H3_FLAG_TEXT_T_ONLY = 1,       /* text at (t, 0, 0) instead of (t, t, t) */
+  H3_FLAG_AUDIO_CHANNEL_H = 2,   /* stereo channel on the h axis instead of w */
+  H3_FLAG_VIDEO_CANVAS = 4       /* reserved: normalised spatial canvas (not implemented) */
+};
+
+/*
+ * One contiguous run of logical elements of one modality ([P1] section 4;
+ * [P3] latent-frame, text and clock passages).
+ *
+ * Logical element order: segments in table order; inside a text segment the
+ * token index i; inside a video segment (frame k, y, x) row-major over a
+ * grid_h x grid_w patch grid; inside an audio segment (token j, channel c).
+ *
+ * Time of element index idx (i, k or j) is the exact rational
+ *     t = (t_off_num + idx * t_step_num) / t_den
+ * in clock units of one audio latent (1/40 s).  A 4x-temporal latent video
+ * frame advances 20/3 units (t_step_num = 20, t_den = 3); audio advances 1.
+ * Coordinates produced (t, h, w):
+ *     text  : (t, t, t), or (t, 0, 0) with H3_FLAG_TEXT_T_ONLY
+ *     video : (t, y, x)
+ *     audio : (t, 0, c), or (t, c, 0) with H3_FLAG_AUDIO_CHANNEL_H
+ * Exactness: |t_off_num + idx * t_step_num| < 2^24 and 0 < t_den < 2^24 for
+ * every idx; then the fp32 value is the correctly rounded quotient.
+ */
+typedef struct {
+  int32_t kind;        /* H3_SEG_TEXT / H3_SEG_VIDEO / H3_SEG_AUDIO */
+  int32_t count;       /* text tokens / latent frames / audio tokens (>= 0) */
+  int32_t grid_h;      /* video: patch-grid height (> 0) */
+  int32_t grid_w;      /* video: patch-grid width  (> 0) */
+  int32_t channels;    /* audio: channels (1 or 2) */
+  int32_t t_off_num;
+  int32_t t_step_num;
+  int32_t t_den;       /* > 0 */
+  int32_t flags;       /* H3_FLAG_* */
+} h3_segment;
+
+#define H3_MAX_SEGMENTS 64
+
+/*
+ * Rotary configuration ([P3] rope-config passage; [P5] H3-Omni-Transformer).
+ * The head dimension is split into per-axis sections sec_t + sec_h + sec_w
+ * == head_dim (each even); axis a with D_a dims rotates D_a/2 pairs with
+ * inverse frequencies theta^(-2j / D_a), j = 0 .. D_a/2 - 1, computed in fp64.
+ * pair_layout 0: pair p = dims (2p, 2p+1); pairs [0, sec_t/2) are t, then h,
+ * then w.  pair_layout 1: pair p = dims (p, p + head_dim/2), same axis order.
+ * A pair (x0, x1) at angle a becomes (x0 cos a - x1 sin a, x0 sin a + x1 cos a).
+ */
+typedef struct {
+  double theta;        /* rotary base, > 1 (10000) */
+  int32_t head_dim;    /* must be 128 */
+  int32_t sec_t;       /* 32 */
+  int32_t sec_h;       /* 48 */
+  int32_t sec_w;       /* 48 */
+  int32_t pair_layout; /* 0 (adjacent, default) or 1 (half-split) */
+} h3_rope_cfg;
+
+/* Short English text for a status code (static storage; never NULL). */
+const char* h3_status_str(int32_t status);
+
+/* Library ABI version (major * 100 + minor). */
+int32_t h3_version(void);
+
+/*
+ * h3_build_coords -- packed segment table -> per-row (t, h, w) fp32.
+ * Defining passages: [P1] section 4 (three axes, shared timeline, stereo
+ * channel on another axis, row order carries no position); [P3] latent-frame,
+ * text and clock-unit passages.
+ *
+ *   segs     host array of nseg segments (1 <= nseg <= H3_MAX_SEGMENTS)
+ *   d_perm   device int32[n_rows]: packed row r holds logical element
+ *            d_perm[r]; NULL = identity.  Entries outside [0, n_rows) are
+ *            reported as H3_ERR_DEVICE_INPUT by h3_check_device_error and
+ *            their rows get NaN coordinates.  That d_perm is a permutation
+ *            is the caller's responsibility.
+ *   n_rows   sum of the segments' rows (else H3_ERR_INVALID_ARG); 0 is allowed
+ *   d_coords device float[n_rows][3], written
+ * Errors: H3_ERR_INVALID_ARG for a bad table (unknown kind or flag, negative
+ * count, non-positive grid/channels/t_den, values outside the exact range),
+ * a row-count mismatch or a NULL d_coords with n_rows > 0.
+ */
+h3_status h3_build_coords(const h3_segment* segs, int32_t nseg, const int32_t* d_perm,
+                          int64_t n_rows, float* d_coords, void* stream);
+
+/*
+ * h3_mmrope_qk -- rotate Q and K in one pass (three-axis MM-RoPE).
+ * Defining passages: [P1] section 4; [P3] chain from the frame rescale to the
+ * position grid to rotate(Q, K); [P5] H3-Omni-Transformer.
+ *
+ *   d_q, d_k          device bf16 inputs, layout above (batch folded into rows)
+ *   d_q_out, d_k_out  device bf16 outputs, same layout and stride; may equal
+ *                     the inputs (in place); must not partially overlap them
+ *   d_coords          device float[n_rows][3] from h3_build_coords
+ *   n_rows, n_heads   rows and heads; row_stride in elements
+ *   cfg               host rotary configuration
+ * Per element: the rotation is computed in fp32 from fp32 cos/sin of an fp64
+ * angle (fp64 coordinate x fp64 inverse frequency), rounded to bf16 (RNE).
+ * Errors: H3_ERR_INVALID_ARG (NULL pointer with n_rows > 0, bad cfg, bad
+ * sizes); H3_ERR_UNSUPPORTED (head_dim != 128, stride not a multiple of 8,
+ * pointer not 16-byte aligned).
+ */
+h3_status h3_mmrope_qk(const void* d_q, const void* d_k, void* d_q_out, void* d_k_out,
+                       const float* d_coords, int64_t n_rows, int32_t n_heads,
+                       int64_t row_stride, const h3_rope_cfg* cfg, void* stream);
+
+/*
+ * h3_packed_attention -- full (non-causal, unmasked) softmax attention over
+ * all packed rows, per batch and head:  O = softmax(Q K^T * scale) V.
+ * Defining passages: [P1] sections 2 and 6 (one packed sequence, full
+ * attention); [P3] bidirectional-attention passage.
+ *
+ *   d_q, d_k, d_v   device bf16 [batch][n_rows][n_heads][128] (Q, K already
+ *                   rotated when d_coords is NULL)
+ *   d_o             device bf16 output, same layout and row_stride
+ *   d_lse           device float[batch][n_heads][n_rows] natural-log row
+ *                   log-sum-exp of the scaled logits, or NULL
+ *   d_coords, cfg   must be NULL: rotation fused into the tile load is not
+ *                   available in this version (H3_ERR_UNSUPPORTED)
+ *   softmax_scale   > 0, or <= 0 for 1/sqrt(head_dim)
+ * Arithmetic: bf16 tensor-core products with fp32 accumulation (tcgen05),
+ * fp32 online softmax, P rounded to bf16 for the P.V product, O rounded to
+ * bf16.  All waits inside the kernel are bounded; on expiry the kernel stops
+ * and h3_check_device_error returns H3_ERR_TIMEOUT.
+ * Errors: H3_ERR_INVALID_ARG (NULL pointers with n_rows > 0, n_rows >= 2^31,
+ * batch or n_heads < 1, bad stride); H3_ERR_UNSUPPORTED (head_dim != 128,
+ * misaligned pointer or stride, d_coords != NULL).
+ */
+h3_status h3_packed_attention(const void* d_q, const void* d_k, const void* d_v, void* d_o,
+                              float* d_lse, const float* d_coords, const h3_rope_cfg* cfg,
+                              int32_t batch, int64_t n_rows, int32_t n_heads, int32_t head_dim,
+                              int64_t row_stride, float softmax_scale, void* stream);
+
+/*
+ * Synchronise `stream`, then read and clear this device's error word.
+ * Returns H3_OK, H3_ERR_TIMEOUT, H3_ERR_DEVICE_INPUT or H3_ERR_CUDA.
+ */
+h3_status h3_check_device_error(void* stream);
+
+/*
+ * Limit, in nanoseconds of device global time, of every bounded wait inside
+ * the attention kernel (process-wide; default 2e9 = 2 s).  0 restores the
+ * default.  Used by tests to force the timeout path.
+ */
+h3_status h3_set_wait_limit_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* H3_H_ */

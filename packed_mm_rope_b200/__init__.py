@@ -1,0 +1,107 @@
+"""packed_mm_rope_b200 -- packed multimodal MM-RoPE attention for B200 (sm_100a).
+
+Thin Python layer over the C ABI of ``libh3.so`` (include/h3.h).  PyTorch is
+used only to hold device memory and to name the current CUDA stream; every
+step of the path runs in the library's CUDA kernels:
+
+* ``h3_build_coords``     packed segment table -> per-row (t, h, w) fp32
+* ``h3_mmrope_qk``        three-axis rotary rotation of bf16 Q and K
+* ``h3_packed_attention`` full softmax attention over the packed rows
+
+Importing the package loads the library and raises if it is missing; there is
+no CPU or eager-PyTorch fallback.
+"""
+from __future__ import annotations
+
+from . import _lib
+from ._lib import (H3Error, H3_OK, H3_ERR_INVALID_ARG, H3_ERR_UNSUPPORTED, H3_ERR_CUDA,  # noqa: F401
+                   H3_ERR_TIMEOUT, H3_ERR_DEVICE_INPUT, h3_build_coords, h3_check_device_error,
+                   h3_mmrope_qk, h3_packed_attention, h3_set_wait_limit_ns, rope_cfg, status_str)
+
+LIB = _lib.load()
+
+
+def _stream(stream=None) -> int:
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _row_layout(x):
+    """(batch, n_rows, n_heads, row_stride) of a [.., N, H, 128] bf16 view."""
+    import torch
+    if x.dtype != torch.bfloat16 or not x.is_cuda:
+        raise TypeError("expected a CUDA bf16 tensor")
+    if x.dim() not in (3, 4) or x.shape[-1] != 128 or x.stride(-1) != 1 or x.stride(-2) != 128:
+        raise ValueError("expected [N, H, 128] or [B, N, H, 128] with heads contiguous")
+    n, h = x.shape[-3], x.shape[-2]
+    rs = x.stride(-3)
+    b = x.shape[0] if x.dim() == 4 else 1
+    if x.dim() == 4 and b > 1 and x.stride(0) != n * rs:
+        raise ValueError("batch stride must be n_rows * row_stride")
+    return b, n, h, rs
+
+
+def build_coords(segments, n_rows: int, perm=None, out=None, stream=None):
+    """fp32 [n_rows, 3] coordinates on the current device."""
+    import torch
+    if out is None:
+        out = torch.empty((n_rows, 3), dtype=torch.float32, device="cuda")
+    p = 0
+    if perm is not None:
+        if perm.dtype != torch.int32 or not perm.is_cuda or perm.numel() != n_rows:
+            raise ValueError("perm must be a CUDA int32 tensor of n_rows entries")
+        p = perm.data_ptr()
+    h3_build_coords(segments, p, n_rows, out.data_ptr(), _stream(stream))
+    return out
+
+
+def mmrope_qk(q, k, coords, q_out=None, k_out=None, theta=10000.0, sections=(32, 48, 48), pair_layout=0,
+              stream=None):
+    """Rotate Q and K; returns (q_out, k_out).  Pass q_out=q, k_out=k for in place."""
+    import torch
+    b, n, h, rs = _row_layout(q)
+    if _row_layout(k) != (b, n, h, rs):
+        raise ValueError("q and k layouts differ")
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    if _row_layout(q_out) != (b, n, h, rs) or _row_layout(k_out) != (b, n, h, rs):
+        raise ValueError("outputs must share the inputs' layout")
+    if coords.dtype != torch.float32 or coords.numel() != 3 * b * n or not coords.is_contiguous():
+        raise ValueError("coords must be contiguous fp32 [rows, 3]")
+    h3_mmrope_qk(q.data_ptr(), k.data_ptr(), q_out.data_ptr(), k_out.data_ptr(), coords.data_ptr(), b * n, h,
+                 rs, rope_cfg(theta, 128, sections, pair_layout), _stream(stream))
+    return q_out, k_out
+
+
+def packed_attention(q, k, v, out=None, lse=None, softmax_scale: float = 0.0, stream=None):
+    """O = softmax(Q K^T * scale) V over all packed rows, per head."""
+    import torch
+    lay = _row_layout(q)
+    if _row_layout(k) != lay or _row_layout(v) != lay:
+        raise ValueError("q, k, v layouts differ")
+    out = torch.empty_like(q) if out is None else out
+    if _row_layout(out) != lay:
+        raise ValueError("output must share the inputs' layout")
+    b, n, h, rs = lay
+    lp = 0
+    if lse is not None:
+        if lse.dtype != torch.float32 or lse.numel() != b * h * n or not lse.is_contiguous():
+            raise ValueError("lse must be contiguous fp32 [B, H, N]")
+        lp = lse.data_ptr()
+    h3_packed_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lp, b, n, h, rs,
+                        softmax_scale, stream=_stream(stream))
+    return out
+
+
+def packed_mmrope_attention(segments, q, k, v, perm=None, theta=10000.0, sections=(32, 48, 48),
+                            pair_layout=0, out=None, lse=None, softmax_scale: float = 0.0, stream=None):
+    """The whole path on one packed sequence: coords -> rotate Q, K -> attention.
+
+    q, k, v: [N, H, 128] bf16 on the GPU (unrotated).  Returns O [N, H, 128].
+    """
+    import torch
+    n = q.shape[-3]
+    coords = build_coords(segments, n, perm, stream=stream)
+    qr, kr = mmrope_qk(q, k, coords, theta=theta, sections=sections, pair_layout=pair_layout, stream=stream)
+    return packed_attention(qr, kr, v, out=out, lse=lse, softmax_scale=softmax_scale, stream=stream)

@@ -1,0 +1,251 @@
+// h3.cu -- the C ABI of libh3 (declared in include/h3.h).
+//
+// Host-side argument validation, TMA tensor-map encoding and kernel launches.
+// The library allocates no device memory; the per-device error word is a
+// static __device__ variable of this module.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "coords.cuh"
+#include "rope.cuh"
+#include "attention.cuh"
+
+namespace {
+
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;   // 2 s per wait
+constexpr uint64_t kDrainLimitNs = 2000000000ull;
+uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n > 0 ? n : 148;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D map over a bf16 [batch][n_rows][row_stride] tensor whose first
+// n_heads*128 columns are used; box = 64 columns x 128 rows, 128-byte swizzle.
+bool make_qkv_map(CUtensorMap* map, const void* ptr, int32_t batch, int64_t n_rows, int32_t n_heads,
+                  int64_t row_stride) {
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(n_heads) * 128u, static_cast<cuuint64_t>(n_rows),
+                              static_cast<cuuint64_t>(batch)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_stride) * 2u,
+                                 static_cast<cuuint64_t>(row_stride) * 2u * static_cast<cuuint64_t>(n_rows)};
+  const cuuint32_t box[3] = {64u, 128u, 1u};
+  const cuuint32_t estride[3] = {1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+                  estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool valid_rope_cfg(const h3_rope_cfg* cfg) {
+  if (cfg == nullptr) return false;
+  if (!(cfg->theta > 1.0) || !std::isfinite(cfg->theta)) return false;
+  if (cfg->sec_t < 0 || cfg->sec_h < 0 || cfg->sec_w < 0) return false;
+  if ((cfg->sec_t | cfg->sec_h | cfg->sec_w) & 1) return false;
+  if (cfg->sec_t + cfg->sec_h + cfg->sec_w != cfg->head_dim) return false;
+  if (cfg->pair_layout != 0 && cfg->pair_layout != 1) return false;
+  return true;
+}
+
+h3::RopeTable make_rope_table(const h3_rope_cfg* cfg) {
+  h3::RopeTable t;
+  const int sec[3] = {cfg->sec_t, cfg->sec_h, cfg->sec_w};
+  int p = 0;
+  for (int a = 0; a < 3; ++a)
+    for (int j = 0; j < sec[a] / 2; ++j, ++p) {
+      t.inv_freq[p] = std::pow(cfg->theta, -2.0 * j / sec[a]);
+      t.axis[p] = a;
+    }
+  return t;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* h3_status_str(int32_t status) {
+  switch (status) {
+    case H3_OK: return "ok";
+    case H3_ERR_INVALID_ARG: return "invalid argument";
+    case H3_ERR_UNSUPPORTED: return "unsupported argument";
+    case H3_ERR_CUDA: return "CUDA error";
+    case H3_ERR_TIMEOUT: return "bounded device wait expired";
+    case H3_ERR_DEVICE_INPUT: return "kernel found an invalid input";
+    default: return "unknown status";
+  }
+}
+
+int32_t h3_version(void) { return 100; }
+
+h3_status h3_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns = ns == 0 ? kDefaultWaitLimitNs : ns;
+  return H3_OK;
+}
+
+h3_status h3_build_coords(const h3_segment* segs, int32_t nseg, const int32_t* d_perm, int64_t n_rows,
+                          float* d_coords, void* stream) {
+  if (segs == nullptr || nseg < 1 || nseg > H3_MAX_SEGMENTS || n_rows < 0) return H3_ERR_INVALID_ARG;
+  static_assert(sizeof(h3::CoordTable) <= 4000, "segment table must fit in kernel parameters");
+  h3::CoordTable tab;
+  std::memset(&tab, 0, sizeof(tab));
+  tab.nseg = nseg;
+  long long first = 0;
+  constexpr long long kExact = 1ll << 24;   // integers below this are exact in fp32
+  for (int i = 0; i < nseg; ++i) {
+    const h3_segment& s = segs[i];
+    if (s.count < 0 || s.t_den <= 0 || s.t_den >= kExact) return H3_ERR_INVALID_ARG;
+    long long rows = 0;
+    if (s.kind == H3_SEG_TEXT) {
+      if (s.flags & ~H3_FLAG_TEXT_T_ONLY) return H3_ERR_INVALID_ARG;
+      rows = s.count;
+    } else if (s.kind == H3_SEG_VIDEO) {
+      if (s.flags != 0) return s.flags == H3_FLAG_VIDEO_CANVAS ? H3_ERR_UNSUPPORTED : H3_ERR_INVALID_ARG;
+      if (s.grid_h <= 0 || s.grid_w <= 0 || s.grid_h >= kExact || s.grid_w >= kExact)
+        return H3_ERR_INVALID_ARG;
+      rows = static_cast<long long>(s.count) * s.grid_h * s.grid_w;
+    } else if (s.kind == H3_SEG_AUDIO) {
+      if (s.flags & ~H3_FLAG_AUDIO_CHANNEL_H) return H3_ERR_INVALID_ARG;
+      if (s.channels < 1 || s.channels > 2) return H3_ERR_INVALID_ARG;
+      rows = static_cast<long long>(s.count) * s.channels;
+    } else {
+      return H3_ERR_INVALID_ARG;
+    }
+    if (s.count > 0) {   // t is linear in the index: check both ends
+      const long long t0 = s.t_off_num;
+      const long long t1 = s.t_off_num + static_cast<long long>(s.count - 1) * s.t_step_num;
+      if (t0 <= -kExact || t0 >= kExact || t1 <= -kExact || t1 >= kExact) return H3_ERR_INVALID_ARG;
+    }
+    tab.seg[i] = s;
+    tab.first[i] = first;
+    first += rows;
+    if (first > (1ll << 40)) return H3_ERR_INVALID_ARG;
+  }
+  tab.first[nseg] = first;
+  if (first != n_rows) return H3_ERR_INVALID_ARG;
+  if (n_rows == 0) return H3_OK;
+  if (d_coords == nullptr) return H3_ERR_INVALID_ARG;
+  const int threads = 256;
+  const long long blocks_needed = (n_rows + threads - 1) / threads;
+  const int blocks = static_cast<int>(blocks_needed < 8LL * sm_count() ? blocks_needed : 8LL * sm_count());
+  h3::coords_kernel<<<blocks, threads, 0, as_stream(stream)>>>(tab, d_perm, n_rows, d_coords);
+  return cudaGetLastError() == cudaSuccess ? H3_OK : H3_ERR_CUDA;
+}
+
+h3_status h3_mmrope_qk(const void* d_q, const void* d_k, void* d_q_out, void* d_k_out,
+                       const float* d_coords, int64_t n_rows, int32_t n_heads, int64_t row_stride,
+                       const h3_rope_cfg* cfg, void* stream) {
+  if (n_rows < 0 || n_heads < 1 || !valid_rope_cfg(cfg)) return H3_ERR_INVALID_ARG;
+  if (cfg->head_dim != 128) return H3_ERR_UNSUPPORTED;
+  if (row_stride < static_cast<int64_t>(n_heads) * 128) return H3_ERR_INVALID_ARG;
+  if (n_rows == 0) return H3_OK;
+  if (!d_q || !d_k || !d_q_out || !d_k_out || !d_coords) return H3_ERR_INVALID_ARG;
+  if (row_stride % 8 != 0 || !aligned16(d_q) || !aligned16(d_k) || !aligned16(d_q_out) ||
+      !aligned16(d_k_out))
+    return H3_ERR_UNSUPPORTED;
+  if (static_cast<long long>(n_heads) * 16 > (1ll << 30)) return H3_ERR_INVALID_ARG;
+  const h3::RopeTable tab = make_rope_table(cfg);
+  const long long nblk = (n_rows + h3::ROPE_ROWS - 1) / h3::ROPE_ROWS;
+  const long long cap = 8LL * sm_count();
+  const int grid = static_cast<int>(nblk < cap ? nblk : cap);
+  const long long stride16 = row_stride / 8;
+  auto q = static_cast<const uint4*>(d_q);
+  auto k = static_cast<const uint4*>(d_k);
+  auto qo = static_cast<uint4*>(d_q_out);
+  auto ko = static_cast<uint4*>(d_k_out);
+  if (cfg->pair_layout == 0)
+    h3::rope_kernel<0><<<grid, h3::ROPE_THREADS, 0, as_stream(stream)>>>(q, k, qo, ko, d_coords, n_rows,
+                                                                       n_heads, stride16, tab);
+  else
+    h3::rope_kernel<1><<<grid, h3::ROPE_THREADS, 0, as_stream(stream)>>>(q, k, qo, ko, d_coords, n_rows,
+                                                                       n_heads, stride16, tab);
+  return cudaGetLastError() == cudaSuccess ? H3_OK : H3_ERR_CUDA;
+}
+
+h3_status h3_packed_attention(const void* d_q, const void* d_k, const void* d_v, void* d_o, float* d_lse,
+                              const float* d_coords, const h3_rope_cfg* cfg, int32_t batch, int64_t n_rows,
+                              int32_t n_heads, int32_t head_dim, int64_t row_stride, float softmax_scale,
+                              void* stream) {
+  (void)cfg;
+  if (batch < 1 || n_heads < 1 || n_rows < 0 || n_rows >= (1ll << 31)) return H3_ERR_INVALID_ARG;
+  if (head_dim != 128) return H3_ERR_UNSUPPORTED;
+  if (d_coords != nullptr) return H3_ERR_UNSUPPORTED;
+  if (row_stride < static_cast<int64_t>(n_heads) * 128) return H3_ERR_INVALID_ARG;
+  if (batch > 65535 || n_heads > 65535) return H3_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return H3_ERR_INVALID_ARG;
+  if (n_rows == 0) return H3_OK;
+  if (!d_q || !d_k || !d_v || !d_o) return H3_ERR_INVALID_ARG;
+  if (row_stride % 8 != 0 || !aligned16(d_q) || !aligned16(d_k) || !aligned16(d_v) || !aligned16(d_o))
+    return H3_ERR_UNSUPPORTED;
+  CUtensorMap tq, tk, tv;
+  if (!make_qkv_map(&tq, d_q, batch, n_rows, n_heads, row_stride) ||
+      !make_qkv_map(&tk, d_k, batch, n_rows, n_heads, row_stride) ||
+      !make_qkv_map(&tv, d_v, batch, n_rows, n_heads, row_stride))
+    return H3_ERR_CUDA;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(h3::attn::attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(h3::attn::SMEM_BYTES));
+  });
+  if (attr_err != cudaSuccess) return H3_ERR_CUDA;
+
+  h3::attn::Params p;
+  p.n_rows = static_cast<int>(n_rows);
+  p.n_heads = n_heads;
+  p.n_kv_tiles = static_cast<int>((n_rows + h3::attn::BN - 1) / h3::attn::BN);
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(128.0f);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o = static_cast<__nv_bfloat16*>(d_o);
+  p.o_row_stride = row_stride;
+  p.o_batch_stride = row_stride * n_rows;
+  p.lse = d_lse;
+  p.wait_limit_ns = g_wait_limit_ns;
+  p.drain_limit_ns = kDrainLimitNs;
+  const dim3 grid(static_cast<unsigned>((n_rows + 2 * h3::attn::BM - 1) / (2 * h3::attn::BM)),
+                  static_cast<unsigned>(n_heads), static_cast<unsigned>(batch));
+  h3::attn::attention_kernel<<<grid, h3::attn::THREADS, h3::attn::SMEM_BYTES, as_stream(stream)>>>(tq, tk, tv,
+                                                                                                  p);
+  return cudaGetLastError() == cudaSuccess ? H3_OK : H3_ERR_CUDA;
+}
+
+h3_status h3_check_device_error(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return H3_ERR_CUDA;
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, h3::g_error_word, sizeof(word)) != cudaSuccess) return H3_ERR_CUDA;
+  if (word != 0 && cudaMemcpyToSymbol(h3::g_error_word, &zero, sizeof(zero)) != cudaSuccess)
+    return H3_ERR_CUDA;
+  if (word & h3::DEVERR_TIMEOUT) return H3_ERR_TIMEOUT;
+  if (word & h3::DEVERR_INPUT) return H3_ERR_DEVICE_INPUT;
+  return H3_OK;
+}
+
+}  // extern "C"

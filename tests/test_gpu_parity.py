@@ -1,0 +1,229 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Coordinates must be bit-exact; rotated Q/K within one bf16 ulp (plus fp32
+slack); attention within max |err| <= 2e-2, mean |err| <= 2e-3 and relative
+error <= 1e-2 against the oracle on the same bf16 inputs.  Small workloads
+are compared in full; the three large ones (28,196 / 81,792 / 31,952 rows x
+42 heads) run in full on the GPU in the benchmark's launch configuration and
+are compared on seeded sampled query rows (every segment kind, rows 0 and
+N-1, the whole last partial tile) for four heads.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import workload as W
+from oracle import attention as oattn
+from oracle import coords as ocoords
+from oracle import pipeline as opipe
+from oracle import rope as orope
+from tests.gpu_util import (bf16_bits_to_f64, check_attention, check_rope, from_dev_bf16, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def h3():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import packed_mm_rope_b200 as lib
+    return lib
+
+
+def _perm_dev(perm):
+    return None if perm is None else torch.from_numpy(perm.astype(np.int32)).cuda()
+
+
+def _sync_ok(h3):
+    st = h3.h3_check_device_error()
+    assert st == h3.H3_OK, h3.status_str(st)
+
+
+# ------------------------------------------------------------ coordinates --
+
+@pytest.mark.parametrize("cfg", range(5))
+def test_coords_bit_exact(h3, cfg):
+    wl = W.workload(cfg)
+    perm = W.permutation(wl)
+    got = h3.build_coords(wl.segments, wl.n_rows, _perm_dev(perm)).cpu().numpy()
+    _sync_ok(h3)
+    num, den = ocoords.packed_coords(wl.segments, perm)
+    want = ocoords.to_f32(num, den)
+    assert got.dtype == np.float32 and got.shape == want.shape
+    assert got.tobytes() == want.tobytes()
+
+
+def test_coords_flags_and_odd_tables(h3):
+    segs = [W.text(5, flags=W.FLAG_TEXT_T_ONLY), W.audio(3, 2, t_off=-7, flags=W.FLAG_AUDIO_CHANNEL_H),
+            W.Segment(W.SEG_TEXT, 0), W.video(3, 2, 3, t_off_num=-1), W.audio(4, 1, t_off=100),
+            W.Segment(W.SEG_VIDEO, 2, 1, 1, 0, 5, 7, 11), W.Segment(W.SEG_VIDEO, 0, 4, 4)]
+    n = sum(s.rows for s in segs)
+    perm = W.fisher_yates(n, 99)
+    for p in (None, perm):
+        got = h3.build_coords(segs, n, _perm_dev(p)).cpu().numpy()
+        _sync_ok(h3)
+        num, den = ocoords.packed_coords(segs, p)
+        assert got.tobytes() == ocoords.to_f32(num, den).tobytes()
+
+
+def test_coords_reject_out_of_range_perm(h3):
+    segs = [W.text(10)]
+    perm = np.arange(10, dtype=np.int32)
+    perm[3] = 10
+    out = h3.build_coords(segs, 10, _perm_dev(perm)).cpu().numpy()
+    assert h3.h3_check_device_error() == h3.H3_ERR_DEVICE_INPUT
+    assert np.isnan(out[3]).all() and np.isfinite(np.delete(out, 3, axis=0)).all()
+    assert h3.h3_check_device_error() == h3.H3_OK      # the word was cleared
+
+
+# ------------------------------------------------------------------- rope --
+
+def _rope_case(h3, wl, rows=None, pair_layout=0, in_place=False):
+    perm = W.permutation(wl)
+    q, k, _ = W.qkv_bf16(wl)
+    coords = h3.build_coords(wl.segments, wl.n_rows, _perm_dev(perm))
+    qd, kd = to_dev(q), to_dev(k)
+    if in_place:
+        qo, ko = h3.mmrope_qk(qd, kd, coords, q_out=qd, k_out=kd, pair_layout=pair_layout)
+    else:
+        qo, ko = h3.mmrope_qk(qd, kd, coords, pair_layout=pair_layout)
+    _sync_ok(h3)
+    rows = np.arange(wl.n_rows) if rows is None else rows
+    num, den = ocoords.packed_coords(wl.segments, perm)
+    ang = orope.angles(ocoords.to_f64(num, den)[rows], wl.theta, wl.sections)
+    res = []
+    for x_bits, out in ((q, qo), (k, ko)):
+        x = bf16_bits_to_f64(x_bits[rows])
+        exact = orope.rotate(x, ang, pair_layout)
+        got = from_dev_bf16(out)[rows]
+        res.append(check_rope(got, exact, x, pair_layout))
+    return res
+
+
+@pytest.mark.parametrize("cfg", [0, 1])
+def test_rope_parity_full(h3, cfg):
+    # the ulp bound (plus fp32 slack near cancellation) is asserted inside check_rope
+    for frac_rne, _ in _rope_case(h3, W.workload(cfg)):
+        assert frac_rne > 0.99
+
+
+def test_rope_half_split_and_in_place(h3):
+    for frac_rne, _ in _rope_case(h3, W.workload(1), pair_layout=1):
+        assert frac_rne > 0.99
+    for frac_rne, _ in _rope_case(h3, W.workload(0), in_place=True):
+        assert frac_rne > 0.99
+
+
+def test_rope_parity_worked_example_sampled(h3):
+    wl = W.workload(2)
+    for frac_rne, _ in _rope_case(h3, wl, rows=W.sample_rows(wl, 200)):
+        assert frac_rne > 0.99
+
+
+# -------------------------------------------------------------- attention --
+
+def _random_bf16(shape, seed, scale=1.0):
+    return W.normal_bf16(seed, 0, shape, scale)
+
+
+@pytest.mark.parametrize("n", [1, 2, 100, 127, 128, 129, 255, 256, 257, 383, 600])
+def test_attention_edge_sizes(h3, n):
+    H = 2
+    q, k, v = (_random_bf16((n, H, 128), 50 + n + 7 * i) for i in range(3))
+    lse = torch.empty((1, H, n), dtype=torch.float32, device="cuda")
+    o = h3.packed_attention(to_dev(q), to_dev(k), to_dev(v), lse=lse)
+    _sync_ok(h3)
+    o_ref, lse_ref = oattn.attention(*(bf16_bits_to_f64(a) for a in (q, k, v)))
+    check_attention(bf16_bits_to_f64(from_dev_bf16(o)), o_ref, f"n={n}")
+    np.testing.assert_allclose(lse.cpu().numpy()[0], lse_ref, rtol=0, atol=2e-3)
+
+
+def test_attention_batch_and_fused_qkv_stride(h3):
+    B, N, H = 2, 300, 3
+    qkv = _random_bf16((B, N, 3, H, 128), 77)           # fused projection output layout
+    dev = to_dev(qkv)
+    q, k, v = dev[:, :, 0], dev[:, :, 1], dev[:, :, 2]
+    out = torch.zeros((B, N, 3, H, 128), dtype=torch.bfloat16, device="cuda")
+    o = h3.packed_attention(q, k, v, out=out[:, :, 0])
+    _sync_ok(h3)
+    assert (out[:, :, 1:] == 0).all(), "writes stayed inside the output view"
+    x = bf16_bits_to_f64(qkv)
+    got = bf16_bits_to_f64(from_dev_bf16(o))
+    for b in range(B):
+        o_ref, _ = oattn.attention(x[b, :, 0], x[b, :, 1], x[b, :, 2])
+        check_attention(got[b], o_ref, f"batch {b}")
+
+
+def test_attention_running_max_rescale(h3):
+    # keys of the last tile are scaled so every row's maximum jumps late
+    N, H = 600, 2
+    q = _random_bf16((N, H, 128), 201)
+    k = _random_bf16((N, H, 128), 202)
+    k[512:] = W.bf16_bits_rne(bf16_bits_to_f64(k[512:]) * 6.0)
+    v = _random_bf16((N, H, 128), 203)
+    o = h3.packed_attention(to_dev(q), to_dev(k), to_dev(v))
+    _sync_ok(h3)
+    o_ref, _ = oattn.attention(*(bf16_bits_to_f64(a) for a in (q, k, v)))
+    check_attention(bf16_bits_to_f64(from_dev_bf16(o)), o_ref, "late max")
+
+
+def test_attention_softmax_scale(h3):
+    N, H = 333, 1
+    q, k, v = (_random_bf16((N, H, 128), 300 + i) for i in range(3))
+    o = h3.packed_attention(to_dev(q), to_dev(k), to_dev(v), softmax_scale=0.25)
+    _sync_ok(h3)
+    o_ref, _ = oattn.attention(*(bf16_bits_to_f64(a) for a in (q, k, v)), scale=0.25)
+    check_attention(bf16_bits_to_f64(from_dev_bf16(o)), o_ref, "scale 0.25")
+
+
+# --------------------------------------------------------- the whole path --
+
+def _pipeline(h3, wl, q, k, v):
+    perm = W.permutation(wl)
+    o = h3.packed_mmrope_attention(wl.segments, to_dev(q), to_dev(k), to_dev(v), perm=_perm_dev(perm),
+                                   theta=wl.theta, sections=wl.sections)
+    _sync_ok(h3)
+    return perm, bf16_bits_to_f64(from_dev_bf16(o))
+
+
+@pytest.mark.parametrize("cfg", [0, 1])
+def test_pipeline_parity_full(h3, cfg):
+    wl = W.workload(cfg)
+    q, k, v = W.qkv_bf16(wl)
+    perm, got = _pipeline(h3, wl, q, k, v)
+    ref, _ = opipe.packed_mmrope_attention(wl.segments, perm, q, k, v, wl.theta, wl.sections)
+    check_attention(got, ref, wl.name)
+
+
+def test_pipeline_peaky_queries(h3):
+    wl = W.workload(1)
+    q, k, v = W.qkv_bf16(wl, q_scale=4.0)
+    perm, got = _pipeline(h3, wl, q, k, v)
+    ref, _ = opipe.packed_mmrope_attention(wl.segments, perm, q, k, v, wl.theta, wl.sections)
+    check_attention(got, ref, "peaky x4")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("cfg", [2, 3, 4])
+def test_pipeline_parity_full_size_sampled(h3, cfg):
+    wl = W.workload(cfg)
+    q, k, v = W.qkv_bf16(wl)
+    perm, got = _pipeline(h3, wl, q, k, v)
+    rows = W.sample_rows(wl, 96)
+    heads = sorted({0, 1, wl.heads // 2, wl.heads - 1})
+    ref, _ = opipe.packed_mmrope_attention(wl.segments, perm, q, k, v, wl.theta, wl.sections,
+                                           rows=rows, heads=heads)
+    check_attention(got[rows][:, heads], ref, wl.name)
+
+
+def test_row_order_carries_no_position_on_gpu(h3):
+    wl = W.workload(0)
+    q, k, v = W.qkv_bf16(wl)
+    perm, got = _pipeline(h3, wl, q, k, v)
+    inv = np.empty_like(perm)
+    inv[perm] = np.arange(perm.size)
+    o = h3.packed_mmrope_attention(wl.segments, to_dev(q[inv]), to_dev(k[inv]), to_dev(v[inv]))
+    _sync_ok(h3)
+    unshuffled = bf16_bits_to_f64(from_dev_bf16(o))
+    assert np.abs(got - unshuffled[perm]).max() <= 2e-2

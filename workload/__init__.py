@@ -139,6 +139,15 @@ def workload(i: int) -> Workload:
     return WORKLOADS[i]
 
 
+def worked_example_resized(frames: int) -> Workload:
+    """The worked-example layout (512 text rows, 22 x 40 latent frames, stereo
+    audio, 42 x 128 heads) with ``frames`` latent frames and ceil(20 * frames / 3)
+    audio tokens -- smaller or larger variants for profiling."""
+    tokens = -(-20 * frames // 3)
+    return Workload(f"worked_example_{frames}f", 2, 42, 128,
+                    (text(512), video(frames, 22, 40), audio(tokens, 2)), shuffle=False)
+
+
 # --------------------------------------------------------------- SplitMix64 --
 
 GAMMA = np.uint64(0x9E3779B97F4A7C15)
