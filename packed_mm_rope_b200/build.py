@@ -44,7 +44,9 @@ def up_to_date() -> bool:
 def build_library(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"),
+    # H3_NVCC_DEFINES="-DNAME=VALUE ..." passes tuning macros (e.g. H3_EXP2_FMA_EVERY)
+    extra = os.environ.get("H3_NVCC_DEFINES", "").split()
+    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"),
            os.path.join(HERE, "csrc", "h3.cu"), "-o", LIB + ".tmp"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:

@@ -16,7 +16,9 @@
 //   [128,256)  S1 = Q1 K_j^T     its first 64 columns, two per column)
 //   [256,384)  O0 accumulator   [384,512) O1 accumulator
 // Per KV tile j the issuer runs  PV0(j), S0(j+1), PV1(j), S1(j+1): while one
-// warpgroup exponentiates its S tile the tensor core works on the other.
+// warpgroup exponentiates its S tile the tensor core works on the other.  Each
+// P tile is released in two 64-key halves with their own barriers, so the
+// first half of P.V runs while the second half is still being exponentiated.
 //
 // Softmax (one thread = one query row, the row lives in one TMEM lane):
 // logits are handled in log2 units (x = s * scale * log2 e).  The running
@@ -24,9 +26,12 @@
 // exceeds it by more than RESCALE_LOG2 (= 8): then O (in TMEM) and the row
 // sum are multiplied by 2^(m_old - m_new).  Otherwise numerators stay <= 2^8,
 // which bf16 and fp32 hold exactly in range; the final O / l is the same
-// quotient either way.  The S tile of step j+1 is only issued after PV(j), so
-// when a warpgroup sees S(j) complete, O already holds all of PV(j-1) and the
-// rescale can be applied in place before P(j) is released.
+// quotient either way.  The check is made per 64-key half, speculatively: the
+// numerators are computed against the current m and kept unless the half's
+// own maximum exceeds it by more than 8.  The S tile of step j+1 is only
+// issued after PV(j), so when a warpgroup sees S(j) complete, O already holds
+// PV(j-1) and a rescale for the first half can be applied in place; a rescale
+// for the second half first waits for the first half of PV(j) to land.
 //
 // Shared memory (1024-byte aligned): Q0, Q1 (32 KB each) and a ring of
 // KV_STAGES 32 KB slots; every 128 x 128 bf16 tile is two 128-row x 64-column
@@ -55,8 +60,9 @@ constexpr float RESCALE_LOG2 = 8.0f;
 constexpr uint32_t SMEM_Q = 0;
 constexpr uint32_t SMEM_KV = 2 * TILE_BYTES;
 constexpr uint32_t SMEM_BAR = SMEM_KV + KV_STAGES * TILE_BYTES;
-// barriers: q_full[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], mma_done
-constexpr int NUM_BARS = 2 + 2 * KV_STAGES + 2 + 2 + 2 + 1;
+// barriers: q_full[2], kv_full[S], kv_empty[S], s_full[2], p_full[2][2] (halves),
+//           pva_done[2] (first half of PV landed), o_full[2], mma_done
+constexpr int NUM_BARS = 2 + 2 * KV_STAGES + 2 + 4 + 2 + 2 + 1;
 constexpr uint32_t SMEM_MISC = SMEM_BAR + NUM_BARS * 8;   // tmem base, abort flag
 constexpr uint32_t SMEM_BYTES = SMEM_MISC + 16 + 1024;    // + alignment slack
 
@@ -65,6 +71,36 @@ constexpr uint32_t IDESC_O = idesc_bf16_f32(BM, HD, false, true);    // P from T
 
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_S0 = 0, TMEM_O0 = 256;
+
+// Every EXP2_FMA_EVERY-th pair of exponentials is computed on the FMA pipe
+// (0 = all on the MUFU unit).  The MUFU unit issues 16 exponentials per clock
+// per SM, the same time the tensor core needs for a 128 x 128 x 128 tile pair,
+// so moving a share of them to the FMA pipe takes the unit off the critical path.
+#ifndef H3_EXP2_FMA_EVERY
+#define H3_EXP2_FMA_EVERY 0
+#endif
+constexpr int EXP2_FMA_EVERY = H3_EXP2_FMA_EVERY;
+
+// 2^x on the FMA pipe: x = n + f with n = nearest integer (the 1.5 * 2^23
+// rounding trick), 2^f by a degree-3 polynomial whose coefficients minimise the
+// maximum RELATIVE error on [-1/2, 1/2] (Remez exchange; fit_exp2_poly.py
+// regenerates them; max relative error 7.5e-5, below bf16's 2^-9 rounding of
+// P), and 2^n added to the exponent field.  x is clamped below at -126 so the
+// exponent stays in range; values that small are zero at bf16 resolution.
+constexpr float EXP2_C0 = 0.9999280571937561f;
+constexpr float EXP2_C1 = 0.6932609677314758f;
+constexpr float EXP2_C2 = 0.2426111251115799f;
+constexpr float EXP2_C3 = 0.0551716685295105f;
+
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -126.f);
+  const float j = __fadd_rn(x, 12582912.f);      // 1.5 * 2^23 + round(x)
+  const float f = __fsub_rn(x, __fsub_rn(j, 12582912.f));
+  float p = fmaf(EXP2_C3, f, EXP2_C2);
+  p = fmaf(p, f, EXP2_C1);
+  p = fmaf(p, f, EXP2_C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(j) << 23));
+}
 
 // All lanes wait; the warp proceeds only if every lane saw the phase complete,
 // so the .sync.aligned tcgen05 instructions that follow run converged.
@@ -87,6 +123,34 @@ struct Params {
   unsigned long long drain_limit_ns;
 };
 
+// 2^(x*sl2 - m) for 64 logits: bf16 pairs, their sum, and the raw maximum.
+// Eight independent accumulators keep the max and sum chains short; every
+// EXP2_FMA_EVERY-th pair is evaluated on the FMA pipe instead of MUFU.
+__device__ __forceinline__ void exp_half(const float (&x)[64], float sl2, float m, uint32_t (&pk)[32],
+                                         float& mx, float& ls) {
+  float ma[8], la[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) { ma[i] = -INFINITY; la[i] = 0.f; }
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    const float x0 = x[2 * c], x1 = x[2 * c + 1];
+    ma[c & 7] = fmaxf(ma[c & 7], fmaxf(x0, x1));
+    const float y0 = fmaf(x0, sl2, -m), y1 = fmaf(x1, sl2, -m);
+    float p0, p1;
+    if (EXP2_FMA_EVERY > 0 && (c % EXP2_FMA_EVERY) == EXP2_FMA_EVERY - 1) {
+      p0 = exp2_fma(y0);
+      p1 = exp2_fma(y1);
+    } else {
+      p0 = ex2_approx(y0);
+      p1 = ex2_approx(y1);
+    }
+    la[c & 7] += p0 + p1;
+    pk[c] = pack_bf16x2(p0, p1);
+  }
+  mx = fmaxf(fmaxf(fmaxf(ma[0], ma[1]), fmaxf(ma[2], ma[3])), fmaxf(fmaxf(ma[4], ma[5]), fmaxf(ma[6], ma[7])));
+  ls = ((la[0] + la[1]) + (la[2] + la[3])) + ((la[4] + la[5]) + (la[6] + la[7]));
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
 attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -100,9 +164,10 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   auto bar_kv_full = [&](int s) { return bar0 + 8u * (2 + s); };
   auto bar_kv_empty = [&](int s) { return bar0 + 8u * (2 + KV_STAGES + s); };
   auto bar_s_full = [&](int i) { return bar0 + 8u * (2 + 2 * KV_STAGES + i); };
-  auto bar_p_full = [&](int i) { return bar0 + 8u * (4 + 2 * KV_STAGES + i); };
-  auto bar_o_full = [&](int i) { return bar0 + 8u * (6 + 2 * KV_STAGES + i); };
-  const uint32_t bar_mma_done = bar0 + 8u * (8 + 2 * KV_STAGES);
+  auto bar_p_full = [&](int i, int half) { return bar0 + 8u * (4 + 2 * KV_STAGES + 2 * i + half); };
+  auto bar_pva_done = [&](int i) { return bar0 + 8u * (8 + 2 * KV_STAGES + i); };
+  auto bar_o_full = [&](int i) { return bar0 + 8u * (10 + 2 * KV_STAGES + i); };
+  const uint32_t bar_mma_done = bar0 + 8u * (12 + 2 * KV_STAGES);
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gbase + SMEM_MISC);
   volatile uint32_t* const abort_flag = reinterpret_cast<volatile uint32_t*>(gbase + SMEM_MISC + 4);
 
@@ -118,7 +183,9 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_q_full(i), 1);
       mbar_init(bar_s_full(i), 1);
-      mbar_init(bar_p_full(i), 128);
+      mbar_init(bar_p_full(i, 0), 128);
+      mbar_init(bar_p_full(i, 1), 128);
+      mbar_init(bar_pva_done(i), 1);
       mbar_init(bar_o_full(i), 1);
     }
     for (int s = 0; s < KV_STAGES; ++s) {
@@ -189,15 +256,28 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                  smem_desc_sw128(kv_addr(ks) + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
-      // O_i += P_i V : A = P_i from TMEM (8 columns per K=16), B = V MN-major
-      auto issue_pv = [&](int i, int vs, bool acc) {
+      // O_i += P_i V over keys [64*half, 64*half + 64): A = P_i from TMEM (8
+      // columns per K=16 step), B = V rows from shared memory, MN-major
+      auto issue_pv = [&](int i, int vs, int half, bool acc) {
         const uint32_t d = tmem + TMEM_O0 + i * 128;
         const uint32_t a = tmem + TMEM_S0 + i * 128;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int kk = 4 * half + k4;
           mma_ts(d, a + kk * 8, smem_desc_sw128(kv_addr(vs) + kk * 2048, HALF_BYTES, 1024),
                  IDESC_O, (acc || kk > 0) ? 1u : 0u);
         }
+      };
+      // P_i(j) in two halves; the first half's completion is announced on pva_done
+      auto issue_pv_tile = [&](int i, int vs, int j) -> bool {
+        if (!mbar_wait_bounded(bar_p_full(i, 0), j & 1, abort_flag, limit)) return false;
+        tc_fence_after();
+        issue_pv(i, vs, 0, j > 0);
+        tc_commit(bar_pva_done(i));
+        if (!mbar_wait_bounded(bar_p_full(i, 1), j & 1, abort_flag, limit)) return false;
+        tc_fence_after();
+        issue_pv(i, vs, 1, true);
+        return true;
       };
       bool ok = mbar_wait_bounded(bar_q_full(0), 0, abort_flag, limit) &&
                 mbar_wait_bounded(bar_kv_full(0), 0, abort_flag, limit);
@@ -218,9 +298,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int kidx = 2 * j + 2, ks = kidx % KV_STAGES;
         const bool more = j + 1 < nkv;
         if (!mbar_wait_bounded(bar_kv_full(vs), (vidx / KV_STAGES) & 1, abort_flag, limit)) break;
-        if (!mbar_wait_bounded(bar_p_full(0), j & 1, abort_flag, limit)) break;
-        tc_fence_after();
-        issue_pv(0, vs, j > 0);
+        if (!issue_pv_tile(0, vs, j)) break;
         if (more) {
           if (!mbar_wait_bounded(bar_kv_full(ks), (kidx / KV_STAGES) & 1, abort_flag, limit)) break;
           tc_fence_after();
@@ -229,9 +307,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         } else {
           tc_commit(bar_o_full(0));
         }
-        if (!mbar_wait_bounded(bar_p_full(1), j & 1, abort_flag, limit)) break;
-        tc_fence_after();
-        issue_pv(1, vs, j > 0);
+        if (!issue_pv_tile(1, vs, j)) break;
         tc_commit(bar_kv_empty(vs));
         if (more) {
           issue_s(1, ks);
@@ -259,30 +335,90 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     float l_sum = 0.f;
     bool ok = true;
 
+    // registers of two TMEM chunks -> 64 logits; keys past the end -> -inf
+    auto to_logits = [&](const uint32_t (&r)[2][32], int col0, bool last, float (&x)[64]) {
+#pragma unroll
+      for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(r[c >> 5][c & 31]);
+      if (last && tail < BN) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (col0 + c >= tail) x[c] = -INFINITY;
+      }
+    };
+    // O *= f for this warp's rows (warp-collective TMEM round trip)
+    auto rescale_o = [&](float f) {
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(t_o + 32 * c, o);
+        tmem_wait_ld(o);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+        tmem_st32(t_o + 32 * c, o);
+      }
+    };
+    // Publish 64 keys of P (32 TMEM columns, aliasing the S columns already read).
+    auto store_p = [&](int half, const uint32_t (&pk)[32]) {
+      __syncwarp();
+      tmem_st32(t_s + 32 * half, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_p_full(wg, half));
+    };
+
     for (int j = 0; j < nkv; ++j) {
       if (!warp_wait(bar_s_full(wg), j & 1, abort_flag, limit)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(t_s + 32 * c, sr[c]);
-      tmem_wait_ld();
-      float s[128];
-#pragma unroll
-      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
-      if (j == nkv - 1 && tail < BN) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= tail) s[c] = -INFINITY;
+      const bool last = j == nkv - 1;
+      float ls_a;
+      {
+        // ---- keys 0..63 ----
+        uint32_t ra[2][32];
+        tmem_ld32(t_s, ra[0]);
+        tmem_ld32(t_s + 32, ra[1]);
+        tmem_wait_ld(ra[0]);
+        tmem_wait_ld(ra[1]);
+        float xa[64];
+        to_logits(ra, 0, last, xa);
+        uint32_t pka[32];
+        float mx;
+        exp_half(xa, sl2, m_used, pka, mx, ls_a);     // speculative against m_used
+        const float m_new = mx * sl2;
+        const bool need = (j == 0) || (m_new > m_used + RESCALE_LOG2);
+        if (__any_sync(0xffffffffu, need)) {
+          float f = 1.f;
+          if (need) {
+            f = (j == 0) ? 0.f : ex2_approx(m_used - m_new);
+            m_used = m_new;
+            l_sum *= f;
+          }
+          __syncwarp();
+          if (j > 0) rescale_o(f);      // O holds PV(j-1); PV(j) has not started
+          exp_half(xa, sl2, m_used, pka, mx, ls_a);
+        }
+        l_sum += ls_a;
+        store_p(0, pka);
       }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
-      const float m_new = mx * sl2;
-      if (j == 0) {
-        m_used = m_new;
-      } else {
+      {
+        // ---- keys 64..127 ----
+        uint32_t rb[2][32];
+        __syncwarp();
+        tmem_ld32(t_s + 64, rb[0]);
+        tmem_ld32(t_s + 96, rb[1]);
+        tmem_wait_ld(rb[0]);
+        tmem_wait_ld(rb[1]);
+        float xb[64];
+        to_logits(rb, 64, last, xb);
+        uint32_t pkb[32];
+        float mx, ls_b;
+        exp_half(xb, sl2, m_used, pkb, mx, ls_b);
+        const float m_new = mx * sl2;
         const bool need = m_new > m_used + RESCALE_LOG2;
         if (__any_sync(0xffffffffu, need)) {
+          // the first half of PV(j) may be in flight: let it land, then rescale
+          // O (which now includes it) together with the running sum
+          if (!warp_wait(bar_pva_done(wg), j & 1, abort_flag, limit)) { ok = false; break; }
+          tc_fence_after();
           float f = 1.f;
           if (need) {
             f = ex2_approx(m_used - m_new);
@@ -290,31 +426,12 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             l_sum *= f;
           }
           __syncwarp();
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(t_o + 32 * c, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-            tmem_st32(t_o + 32 * c, o);
-          }
+          rescale_o(f);
+          exp_half(xb, sl2, m_used, pkb, mx, ls_b);
         }
+        l_sum += ls_b;
+        store_p(1, pkb);
       }
-      // numerators, row sum, bf16 pairs into TMEM (P aliases S's first 64 columns)
-      uint32_t pk[2][32];
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2_approx(fmaf(s[2 * c], sl2, -m_used));
-        const float p1 = ex2_approx(fmaf(s[2 * c + 1], sl2, -m_used));
-        l_sum += p0 + p1;
-        pk[c >> 5][c & 31] = pack_bf16x2(p0, p1);
-      }
-      tmem_st32(t_s, pk[0]);
-      tmem_st32(t_s + 32, pk[1]);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar_p_full(wg));
     }
 
     // epilogue: O / l -> bf16 -> global; optional log-sum-exp
@@ -329,7 +446,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         uint32_t o[32];
         __syncwarp();
         tmem_ld32(t_o + 32 * c, o);
-        tmem_wait_ld();
+        tmem_wait_ld(o);
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)

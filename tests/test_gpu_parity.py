@@ -92,12 +92,13 @@ def _rope_case(h3, wl, rows=None, pair_layout=0, in_place=False):
     rows = np.arange(wl.n_rows) if rows is None else rows
     num, den = ocoords.packed_coords(wl.segments, perm)
     ang = orope.angles(ocoords.to_f64(num, den)[rows], wl.theta, wl.sections)
+    ang32 = orope.angles(ocoords.to_f32(num, den)[rows].astype(np.float64), wl.theta, wl.sections)
     res = []
     for x_bits, out in ((q, qo), (k, ko)):
         x = bf16_bits_to_f64(x_bits[rows])
         exact = orope.rotate(x, ang, pair_layout)
         got = from_dev_bf16(out)[rows]
-        res.append(check_rope(got, exact, x, pair_layout))
+        res.append(check_rope(got, exact, x, pair_layout, dang=np.abs(ang32 - ang)))
     return res
 
 
@@ -201,7 +202,8 @@ def test_pipeline_peaky_queries(h3):
     q, k, v = W.qkv_bf16(wl, q_scale=4.0)
     perm, got = _pipeline(h3, wl, q, k, v)
     ref, _ = opipe.packed_mmrope_attention(wl.segments, perm, q, k, v, wl.theta, wl.sections)
-    check_attention(got, ref, "peaky x4")
+    # logits ~ N(0, 16): absolute tolerances scale with the logit magnitude (x4)
+    check_attention(got, ref, "peaky x4", logit_scale=4.0)
 
 
 @pytest.mark.slow
