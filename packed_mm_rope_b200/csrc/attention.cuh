@@ -21,17 +21,20 @@
 // first half of P.V runs while the second half is still being exponentiated.
 //
 // Softmax (one thread = one query row, the row lives in one TMEM lane):
-// logits are handled in log2 units (x = s * scale * log2 e).  The running
-// maximum m used for the exponentials is only raised when a new row maximum
-// exceeds it by more than RESCALE_LOG2 (= 8): then O (in TMEM) and the row
-// sum are multiplied by 2^(m_old - m_new).  Otherwise numerators stay <= 2^8,
-// which bf16 and fp32 hold exactly in range; the final O / l is the same
-// quotient either way.  The check is made per 64-key half, speculatively: the
-// numerators are computed against the current m and kept unless the half's
-// own maximum exceeds it by more than 8.  The S tile of step j+1 is only
-// issued after PV(j), so when a warpgroup sees S(j) complete, O already holds
-// PV(j-1) and a rescale for the first half can be applied in place; a rescale
-// for the second half first waits for the first half of PV(j) to land.
+// logits are handled in log2 units (x = s * scale * log2 e).  Numerators are
+// 2^(x - m) against a running reference m that is only raised when a 64-key
+// half would overflow the headroom: the half's numerators are computed first
+// (speculatively, against the current m) and kept unless their sum exceeds
+// 2^64.  Then the half's true maximum is taken, O (in TMEM) and the row sum
+// are multiplied by 2^(m_old - m_new), and the half is recomputed.  Any m
+// gives the same quotient O / l; the limit only keeps numerators, sums and O
+// far from fp32/bf16 overflow.  In practice m is set by the first half-tile
+// and never moves again, so the hot loop has no max reduction at all: one
+// packed fp32x2 FMA, two MUFU ex2, one packed add and one bf16x2 conversion per
+// pair of logits.  The S tile of step j+1 is only issued after PV(j), so when
+// a warpgroup sees S(j) complete, O already holds PV(j-1) and a rescale for
+// the first half can be applied in place; a rescale for the second half first
+// waits for the first half of PV(j) to land (pva_done).
 //
 // Shared memory (1024-byte aligned): Q0, Q1 (32 KB each) and a ring of
 // KV_STAGES 32 KB slots; every 128 x 128 bf16 tile is two 128-row x 64-column
@@ -51,11 +54,14 @@ namespace attn {
 constexpr int BM = 128;          // query rows per tile (MMA M)
 constexpr int BN = 128;          // key rows per tile  (S MMA N, PV MMA K)
 constexpr int HD = 128;          // head dim
-constexpr int KV_STAGES = 4;
+#ifndef H3_KV_STAGES
+#define H3_KV_STAGES 4
+#endif
+constexpr int KV_STAGES = H3_KV_STAGES;
 constexpr int THREADS = 320;
 constexpr uint32_t TILE_BYTES = BM * HD * 2;     // 32768
 constexpr uint32_t HALF_BYTES = TILE_BYTES / 2;  // 16384
-constexpr float RESCALE_LOG2 = 8.0f;
+constexpr float SUM_LIMIT = 18446744073709551616.0f;   // 2^64
 
 constexpr uint32_t SMEM_Q = 0;
 constexpr uint32_t SMEM_KV = 2 * TILE_BYTES;
@@ -77,9 +83,12 @@ constexpr uint32_t TMEM_S0 = 0, TMEM_O0 = 256;
 // per SM, the same time the tensor core needs for a 128 x 128 x 128 tile pair,
 // so moving a share of them to the FMA pipe takes the unit off the critical path.
 #ifndef H3_EXP2_FMA_EVERY
-#define H3_EXP2_FMA_EVERY 0
+#define H3_EXP2_FMA_EVERY 0   // measured slower at every share on B200
 #endif
 constexpr int EXP2_FMA_EVERY = H3_EXP2_FMA_EVERY;
+#ifndef H3_EXP_F16X2
+#define H3_EXP_F16X2 0
+#endif
 
 // 2^x on the FMA pipe: x = n + f with n = nearest integer (the 1.5 * 2^23
 // rounding trick), 2^f by a degree-3 polynomial whose coefficients minimise the
@@ -100,6 +109,26 @@ __device__ __forceinline__ float exp2_fma(float x) {
   p = fmaf(p, f, EXP2_C1);
   p = fmaf(p, f, EXP2_C0);
   return __int_as_float(__float_as_int(p) + (__float_as_int(j) << 23));
+}
+
+// Waits of the single MMA-issuing thread spin with test_wait (never suspend):
+// it is on the critical path of both query tiles.
+__device__ __forceinline__ bool mma_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
+                                         uint64_t limit) {
+  return mbar_spin_bounded(bar, parity, abort, limit);
+}
+
+// exp2_fma for two values with packed fp32x2 arithmetic (same steps).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  const float2 big = make_float2(12582912.f, 12582912.f);
+  x = make_float2(fmaxf(x.x, -126.f), fmaxf(x.y, -126.f));
+  const float2 j = __fadd2_rn(x, big);
+  const float2 f = __ffma2_rn(__fadd2_rn(j, make_float2(-12582912.f, -12582912.f)), make_float2(-1.f, -1.f), x);
+  float2 q = __ffma2_rn(make_float2(EXP2_C3, EXP2_C3), f, make_float2(EXP2_C2, EXP2_C2));
+  q = __ffma2_rn(q, f, make_float2(EXP2_C1, EXP2_C1));
+  q = __ffma2_rn(q, f, make_float2(EXP2_C0, EXP2_C0));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(j.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(j.y) << 23)));
 }
 
 // All lanes wait; the warp proceeds only if every lane saw the phase complete,
@@ -123,32 +152,42 @@ struct Params {
   unsigned long long drain_limit_ns;
 };
 
-// 2^(x*sl2 - m) for 64 logits: bf16 pairs, their sum, and the raw maximum.
-// Eight independent accumulators keep the max and sum chains short; every
-// EXP2_FMA_EVERY-th pair is evaluated on the FMA pipe instead of MUFU.
+// 2^(x*sl2 - m) for 64 logits: bf16 pairs and their sum.  Two logits per
+// packed fp32x2 FMA and add (Blackwell f32x2 arithmetic) keep the instruction
+// count per element at 2.5: the softmax warps are issue-bound, not MUFU-bound.
 __device__ __forceinline__ void exp_half(const float (&x)[64], float sl2, float m, uint32_t (&pk)[32],
-                                         float& mx, float& ls) {
-  float ma[8], la[8];
+                                         float& ls) {
+  const float2 c2 = make_float2(sl2, sl2), mm = make_float2(-m, -m);
+  float2 acc[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) { ma[i] = -INFINITY; la[i] = 0.f; }
+  for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
-    const float x0 = x[2 * c], x1 = x[2 * c + 1];
-    ma[c & 7] = fmaxf(ma[c & 7], fmaxf(x0, x1));
-    const float y0 = fmaf(x0, sl2, -m), y1 = fmaf(x1, sl2, -m);
+    const float2 y = __ffma2_rn(make_float2(x[2 * c], x[2 * c + 1]), c2, mm);
     float p0, p1;
     if (EXP2_FMA_EVERY > 0 && (c % EXP2_FMA_EVERY) == EXP2_FMA_EVERY - 1) {
-      p0 = exp2_fma(y0);
-      p1 = exp2_fma(y1);
+      const float2 e = exp2_fma2(y);
+      p0 = e.x;
+      p1 = e.y;
     } else {
-      p0 = ex2_approx(y0);
-      p1 = ex2_approx(y1);
+      p0 = ex2_approx(y.x);
+      p1 = ex2_approx(y.y);
     }
-    la[c & 7] += p0 + p1;
+    acc[c & 3] = __fadd2_rn(acc[c & 3], make_float2(p0, p1));
     pk[c] = pack_bf16x2(p0, p1);
   }
-  mx = fmaxf(fmaxf(fmaxf(ma[0], ma[1]), fmaxf(ma[2], ma[3])), fmaxf(fmaxf(ma[4], ma[5]), fmaxf(ma[6], ma[7])));
-  ls = ((la[0] + la[1]) + (la[2] + la[3])) + ((la[4] + la[5]) + (la[6] + la[7]));
+  const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  ls = t.x + t.y;
+}
+
+// Raw maximum of 64 logits (only on the rare rescale path).
+__device__ __forceinline__ float max64(const float (&x)[64]) {
+  float ma[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ma[i] = x[i];
+#pragma unroll
+  for (int c = 8; c < 64; ++c) ma[c & 7] = fmaxf(ma[c & 7], x[c]);
+  return fmaxf(fmaxf(fmaxf(ma[0], ma[1]), fmaxf(ma[2], ma[3])), fmaxf(fmaxf(ma[4], ma[5]), fmaxf(ma[6], ma[7])));
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -270,22 +309,22 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       };
       // P_i(j) in two halves; the first half's completion is announced on pva_done
       auto issue_pv_tile = [&](int i, int vs, int j) -> bool {
-        if (!mbar_wait_bounded(bar_p_full(i, 0), j & 1, abort_flag, limit)) return false;
+        if (!mma_wait(bar_p_full(i, 0), j & 1, abort_flag, limit)) return false;
         tc_fence_after();
         issue_pv(i, vs, 0, j > 0);
         tc_commit(bar_pva_done(i));
-        if (!mbar_wait_bounded(bar_p_full(i, 1), j & 1, abort_flag, limit)) return false;
+        if (!mma_wait(bar_p_full(i, 1), j & 1, abort_flag, limit)) return false;
         tc_fence_after();
         issue_pv(i, vs, 1, true);
         return true;
       };
-      bool ok = mbar_wait_bounded(bar_q_full(0), 0, abort_flag, limit) &&
-                mbar_wait_bounded(bar_kv_full(0), 0, abort_flag, limit);
+      bool ok = mma_wait(bar_q_full(0), 0, abort_flag, limit) &&
+                mma_wait(bar_kv_full(0), 0, abort_flag, limit);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
         tc_commit(bar_s_full(0));
-        ok = mbar_wait_bounded(bar_q_full(1), 0, abort_flag, limit);
+        ok = mma_wait(bar_q_full(1), 0, abort_flag, limit);
       }
       if (ok) {
         tc_fence_after();
@@ -297,10 +336,10 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int vidx = 2 * j + 1, vs = vidx % KV_STAGES;
         const int kidx = 2 * j + 2, ks = kidx % KV_STAGES;
         const bool more = j + 1 < nkv;
-        if (!mbar_wait_bounded(bar_kv_full(vs), (vidx / KV_STAGES) & 1, abort_flag, limit)) break;
+        if (!mma_wait(bar_kv_full(vs), (vidx / KV_STAGES) & 1, abort_flag, limit)) break;
         if (!issue_pv_tile(0, vs, j)) break;
         if (more) {
-          if (!mbar_wait_bounded(bar_kv_full(ks), (kidx / KV_STAGES) & 1, abort_flag, limit)) break;
+          if (!mma_wait(bar_kv_full(ks), (kidx / KV_STAGES) & 1, abort_flag, limit)) break;
           tc_fence_after();
           issue_s(0, ks);
           tc_commit(bar_s_full(0));
@@ -320,7 +359,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       // Drain: all MMAs issued above complete before TMEM is released.
       tc_commit(bar_mma_done);
       volatile uint32_t never = 0u;
-      mbar_wait_bounded(bar_mma_done, 0, &never, p.drain_limit_ns);
+      mma_wait(bar_mma_done, 0, &never, p.drain_limit_ns);
     }
   } else {
     // -------------------------------------------------------- softmax ----
@@ -381,20 +420,19 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         float xa[64];
         to_logits(ra, 0, last, xa);
         uint32_t pka[32];
-        float mx;
-        exp_half(xa, sl2, m_used, pka, mx, ls_a);     // speculative against m_used
-        const float m_new = mx * sl2;
-        const bool need = (j == 0) || (m_new > m_used + RESCALE_LOG2);
+        exp_half(xa, sl2, m_used, pka, ls_a);         // speculative against m_used
+        const bool need = (j == 0) || !(ls_a <= SUM_LIMIT);
         if (__any_sync(0xffffffffu, need)) {
           float f = 1.f;
           if (need) {
+            const float m_new = fmaxf(m_used, max64(xa) * sl2);
             f = (j == 0) ? 0.f : ex2_approx(m_used - m_new);
             m_used = m_new;
             l_sum *= f;
           }
           __syncwarp();
           if (j > 0) rescale_o(f);      // O holds PV(j-1); PV(j) has not started
-          exp_half(xa, sl2, m_used, pka, mx, ls_a);
+          exp_half(xa, sl2, m_used, pka, ls_a);
         }
         l_sum += ls_a;
         store_p(0, pka);
@@ -410,10 +448,9 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         float xb[64];
         to_logits(rb, 64, last, xb);
         uint32_t pkb[32];
-        float mx, ls_b;
-        exp_half(xb, sl2, m_used, pkb, mx, ls_b);
-        const float m_new = mx * sl2;
-        const bool need = m_new > m_used + RESCALE_LOG2;
+        float ls_b;
+        exp_half(xb, sl2, m_used, pkb, ls_b);
+        const bool need = !(ls_b <= SUM_LIMIT);
         if (__any_sync(0xffffffffu, need)) {
           // the first half of PV(j) may be in flight: let it land, then rescale
           // O (which now includes it) together with the running sum
@@ -421,13 +458,14 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           tc_fence_after();
           float f = 1.f;
           if (need) {
+            const float m_new = fmaxf(m_used, max64(xb) * sl2);
             f = ex2_approx(m_used - m_new);
             m_used = m_new;
             l_sum *= f;
           }
           __syncwarp();
           rescale_o(f);
-          exp_half(xb, sl2, m_used, pkb, mx, ls_b);
+          exp_half(xb, sl2, m_used, pkb, ls_b);
         }
         l_sum += ls_b;
         store_p(1, pkb);

@@ -65,6 +65,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe of the phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Like mbar_wait_bounded, but polls with test_wait: the thread is never
+// suspended, so it sees the phase complete within a few cycles.  For waits on
+// the critical path of a single issuing thread.
+__device__ __forceinline__ bool mbar_spin_bounded(uint32_t bar, uint32_t parity,
+                                                  volatile uint32_t* abort, uint64_t limit_ns) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    for (int i = 0; i < 256; ++i)
+      if (mbar_test_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort = 1u;
+      atomicOr(&g_error_word, DEVERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // Wait until the phase with `parity` has completed.  Gives up (returns false)
 // when `*abort` becomes non-zero or after `limit_ns` of global time; in the
 // latter case it raises `*abort` and the device error word.
@@ -225,6 +257,18 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Two 2^x at once on the MUFU unit in fp16: x is rounded to fp16 (at most
+// 2^-9 absolute for |x| <= 8, i.e. 0.14 % in 2^x), results widened to fp32.
+__device__ __forceinline__ float2 ex2_f16x2(float lo, float hi) {
+  uint32_t h, e;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(hi), "f"(lo));
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(h));
+  float2 r;
+  asm("{\n\t.reg .f16 l, u;\n\tmov.b32 {l, u}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, u;\n\t}"
+      : "=f"(r.x), "=f"(r.y) : "r"(e));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -156,17 +156,23 @@ def test_attention_batch_and_fused_qkv_stride(h3):
         check_attention(got[b], o_ref, f"batch {b}")
 
 
-def test_attention_running_max_rescale(h3):
-    # keys of the last tile are scaled so every row's maximum jumps late
+@pytest.mark.parametrize("gain,cols", [(6.0, slice(512, 600)), (40.0, slice(512, 600)),
+                                       (40.0, slice(64, 128)), (200.0, slice(300, 301))])
+def test_attention_running_max_rescale(h3, gain, cols):
+    # keys of a later tile (or of the second half of one) are scaled so every
+    # row's maximum jumps after the running maximum was set: x6 stays inside the
+    # kernel's headroom, x40 and x200 force the rescale (second half, one key)
     N, H = 600, 2
     q = _random_bf16((N, H, 128), 201)
     k = _random_bf16((N, H, 128), 202)
-    k[512:] = W.bf16_bits_rne(bf16_bits_to_f64(k[512:]) * 6.0)
+    k[cols] = W.bf16_bits_rne(bf16_bits_to_f64(k[cols]) * gain)
     v = _random_bf16((N, H, 128), 203)
-    o = h3.packed_attention(to_dev(q), to_dev(k), to_dev(v))
+    lse = torch.empty((1, H, N), dtype=torch.float32, device="cuda")
+    o = h3.packed_attention(to_dev(q), to_dev(k), to_dev(v), lse=lse)
     _sync_ok(h3)
-    o_ref, _ = oattn.attention(*(bf16_bits_to_f64(a) for a in (q, k, v)))
-    check_attention(bf16_bits_to_f64(from_dev_bf16(o)), o_ref, "late max")
+    o_ref, lse_ref = oattn.attention(*(bf16_bits_to_f64(a) for a in (q, k, v)))
+    check_attention(bf16_bits_to_f64(from_dev_bf16(o)), o_ref, f"late max x{gain}")
+    np.testing.assert_allclose(lse.cpu().numpy()[0], lse_ref, rtol=1e-5, atol=2e-3)
 
 
 def test_attention_softmax_scale(h3):
