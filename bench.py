@@ -20,7 +20,6 @@ Prints ONE JSON line on rank 0.
 from __future__ import annotations
 
 import argparse
-import datetime
 import json
 import os
 import statistics
@@ -129,17 +128,16 @@ def run_ours(args):
 
     import packed_mm_rope_b200 as h3
     from packed_mm_rope_b200 import _lib
+    from packed_mm_rope_b200 import dist as hdist
     import workload as W
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = hdist.world_from_env()
     if world != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+        hdist.init("nccl", device=dev, timeout_s=300)
 
     wl = pick_workload(args)
     N, H, D = wl.n_rows, wl.heads, wl.head_dim
@@ -195,16 +193,8 @@ def run_ours(args):
         step()
         ho.copy_(do, non_blocking=True)
 
-    def barrier():
-        if world > 1:
-            dist.barrier(device_ids=[local])
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier = hdist.barrier
+    max_over_ranks = hdist.max_over_ranks
 
     # warm-up
     for _ in range(args.warmup):
@@ -259,7 +249,7 @@ def run_ours(args):
         return
 
     pk, src = peaks()
-    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    value = hdist.weak_scaling_throughput(flops, world, ms_per_step * 1e-3) / 1e12
     attn_tflops = flops / (attn_ms_max * 1e-3) / 1e12
     rope_bytes = 4 * N * H * D * 2 + N * 12
     rope_gbs = rope_bytes / (rope_ms * 1e-3) / 1e9
@@ -295,12 +285,20 @@ def run_ours(args):
 
 
 def profiled_traffic(wl):
-    """DRAM bytes per attention launch from the committed ncu summary, if it matches this workload."""
+    """DRAM bytes per attention launch from the committed ncu summary.
+
+    Only when the summary was taken on this workload AND on the current kernel
+    source (hash match); otherwise null, as the counters no longer apply.
+    """
+    import hashlib
     path = os.path.join(ROOT, "profiles", "attention_traffic.json")
+    src = os.path.join(ROOT, "packed_mm_rope_b200", "csrc", "attention.cuh")
     try:
         with open(path) as f:
             d = json.load(f)
-        if d.get("n_rows") == wl.n_rows and d.get("heads") == wl.heads:
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        if d.get("n_rows") == wl.n_rows and d.get("heads") == wl.heads and d.get("source_sha256_16") == sha:
             return d.get("dram_bytes_per_launch")
     except (OSError, ValueError):
         pass
