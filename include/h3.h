@@ -64,7 +64,7 @@ enum { H3_SEG_TEXT = 0, H3_SEG_VIDEO = 1, H3_SEG_AUDIO = 2 };
 enum {
   H3_FLAG_TEXT_T_ONLY = 1,       /* text at (t, 0, 0) instead of (t, t, t) */
   H3_FLAG_AUDIO_CHANNEL_H = 2,   /* stereo channel on the h axis instead of w */
-  H3_FLAG_VIDEO_CANVAS = 4       /* reserved: normalised spatial canvas (not implemented) */
+  H3_FLAG_VIDEO_CANVAS = 4       /* video (h, w) on the normalised spatial canvas (below) */
 };
 
 /*
@@ -81,7 +81,12 @@ enum {
  * frame advances 20/3 units (t_step_num = 20, t_den = 3); audio advances 1.
  * Coordinates produced (t, h, w):
  *     text  : (t, t, t), or (t, 0, 0) with H3_FLAG_TEXT_T_ONLY
- *     video : (t, y, x)
+ *     video : (t, y, x), or with H3_FLAG_VIDEO_CANVAS
+ *             (t, c(y, grid_h), c(x, grid_w)) where
+ *             c(i, n) = 16 + (i + 1/2 - n/2) * 32 / sqrt(grid_h * grid_w):
+ *             the grid normalised by sqrt(height x width) and centred on
+ *             [0, 32) ([P3] resolution passage), evaluated in fp64 one IEEE
+ *             operation at a time and rounded to fp32
  *     audio : (t, 0, c), or (t, c, 0) with H3_FLAG_AUDIO_CHANNEL_H
  * Exactness: |t_off_num + idx * t_step_num| < 2^24 and 0 < t_den < 2^24 for
  * every idx; then the fp32 value is the correctly rounded quotient.

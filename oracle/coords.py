@@ -14,6 +14,17 @@ Definition followed:
 Each coordinate is held as an exact rational num/den (int64); ``to_f32``
 returns the correctly rounded (round-to-nearest-even) fp32 value of that
 rational, computed with integer arithmetic only.
+
+Normalised spatial canvas (video flag 4), from the [P3] passage on resolution:
+the (h, w) grid is normalised by sqrt(H * W) and centred on [0, 32), so every
+resolution covers the same range and a wide frame spans wider in w than in h
+about the same midpoint.  Reading: cell centres y + 1/2 are measured from the
+grid centre H/2, scaled by 32 / sqrt(H W), and moved to the midpoint 16:
+    h = 16 + (y + 1/2 - H/2) * 32 / sqrt(H W),  w likewise with x and W.
+The square root makes these irrational; ``packed_values`` evaluates them in
+fp64 with the fixed operation order a = y + 0.5; b = a - 0.5 H;
+s = 32 / sqrt(H W); h = 16 + b * s (each step one IEEE operation) and rounds
+to fp32.
 """
 from __future__ import annotations
 
@@ -26,7 +37,7 @@ FLAG_VIDEO_CANVAS = 4
 
 
 def _field(seg, name, idx):
-    return getattr(seg, name) if hasattr(seg, name) else seg[idx]
+    return seg[idx] if isinstance(seg, (tuple, list)) else getattr(seg, name)
 
 
 def _unpack(seg):
@@ -56,7 +67,7 @@ def logical_coords(segments):
                 num[:, 2], d[:, 2] = t, den
         elif kind == SEG_VIDEO:
             if flags & FLAG_VIDEO_CANVAS:
-                raise NotImplementedError("normalised spatial canvas")
+                raise ValueError("canvas coordinates are irrational: use packed_values")
             k, y, x = np.meshgrid(np.arange(count), np.arange(gh), np.arange(gw), indexing="ij")
             k, y, x = (a.reshape(-1).astype(np.int64) for a in (k, y, x))
             num = np.stack([off + k * step, y, x], axis=1)
@@ -130,3 +141,51 @@ def to_f32(num: np.ndarray, den: np.ndarray) -> np.ndarray:
 def to_f64(num: np.ndarray, den: np.ndarray) -> np.ndarray:
     """fp64 value of each exact rational (one correctly rounded division)."""
     return num.astype(np.float64) / den.astype(np.float64)
+
+
+def canvas_f64(idx: np.ndarray, n: int, h: int, w: int) -> np.ndarray:
+    """16 + (idx + 1/2 - n/2) * 32 / sqrt(h w) in fp64, one IEEE operation per step."""
+    a = np.asarray(idx, np.float64) + 0.5
+    b = a - 0.5 * float(n)
+    s = 32.0 / np.sqrt(float(h) * float(w))
+    return 16.0 + b * s
+
+
+def logical_values(segments):
+    """fp64 and fp32 coordinates of every logical element (any flags).
+
+    Rational coordinates: fp64 = one correctly rounded division, fp32 =
+    correctly rounded rational.  Canvas (h, w): fp64 by ``canvas_f64``,
+    fp32 = round-to-nearest of that fp64 value.
+    """
+    f64s, f32s = [], []
+    for seg in segments:
+        kind, count, gh, gw, ch, off, step, den, flags = _unpack(seg)
+        if kind == SEG_VIDEO and flags & FLAG_VIDEO_CANVAS:
+            plain = (kind, count, gh, gw, ch, off, step, den, flags & ~FLAG_VIDEO_CANVAS)
+            num, d = logical_coords([plain])
+            v64 = to_f64(num, d)
+            v32 = to_f32(num, d)
+            y, x = num[:, 1], num[:, 2]
+            v64[:, 1] = canvas_f64(y, gh, gh, gw)
+            v64[:, 2] = canvas_f64(x, gw, gh, gw)
+            v32[:, 1:] = v64[:, 1:].astype(np.float32)
+        else:
+            num, d = logical_coords([seg])
+            v64, v32 = to_f64(num, d), to_f32(num, d)
+        f64s.append(v64)
+        f32s.append(v32)
+    if not f64s:
+        return np.zeros((0, 3)), np.zeros((0, 3), np.float32)
+    return np.concatenate(f64s), np.concatenate(f32s)
+
+
+def packed_values(segments, perm=None):
+    """(fp64, fp32) coordinates per PACKED row (row r takes logical element perm[r])."""
+    v64, v32 = logical_values(segments)
+    if perm is not None:
+        perm = np.asarray(perm, np.int64)
+        if sorted(perm.tolist()) != list(range(v64.shape[0])):
+            raise ValueError("perm is not a permutation of the logical rows")
+        v64, v32 = v64[perm], v32[perm]
+    return v64, v32

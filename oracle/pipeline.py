@@ -24,8 +24,8 @@ def _as_f64(x: np.ndarray) -> np.ndarray:
 
 
 def packed_angles(segments, perm, theta, sections):
-    num, den = _coords.packed_coords(segments, perm)
-    return _rope.angles(_coords.to_f64(num, den), theta, sections)
+    v64, _ = _coords.packed_values(segments, perm)
+    return _rope.angles(v64, theta, sections)
 
 
 def rotated_qk(segments, perm, q, k, theta=10000.0, sections=(32, 48, 48), pair_layout=0):

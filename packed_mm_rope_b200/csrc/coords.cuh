@@ -29,6 +29,18 @@ __device__ __forceinline__ float exact_ratio(long long num, int den) {
   return __fdiv_rn(static_cast<float>(num), static_cast<float>(den));
 }
 
+// Normalised spatial canvas ("MiniMax H3 -- one transformer ...", passage on
+// resolution: the grid is normalised by sqrt(H W) and centred on [0, 32)):
+//   16 + (idx + 1/2 - n/2) * 32 / sqrt(H W)
+// evaluated in fp64 one IEEE operation at a time (explicit _rn intrinsics, so
+// nothing is contracted into an FMA), then rounded to fp32.
+__device__ __forceinline__ float canvas(long long idx, int n, int gh, int gw) {
+  const double a = __dadd_rn(static_cast<double>(idx), 0.5);
+  const double b = __dsub_rn(a, __dmul_rn(0.5, static_cast<double>(n)));
+  const double s = __ddiv_rn(32.0, __dsqrt_rn(__dmul_rn(static_cast<double>(gh), static_cast<double>(gw))));
+  return __double2float_rn(__dadd_rn(16.0, __dmul_rn(b, s)));
+}
+
 __global__ void __launch_bounds__(256) coords_kernel(const CoordTable tab, const int32_t* perm,
                                                      long long n_rows, float* out) {
   const long long step = static_cast<long long>(gridDim.x) * blockDim.x;
@@ -65,9 +77,15 @@ __global__ void __launch_bounds__(256) coords_kernel(const CoordTable tab, const
       const long long k = local / per_frame;
       const long long cell = local - k * per_frame;
       const long long y = cell / s.grid_w;
+      const long long x = cell - y * s.grid_w;
       t = exact_ratio(s.t_off_num + k * s.t_step_num, s.t_den);
-      h = static_cast<float>(y);
-      w = static_cast<float>(cell - y * s.grid_w);
+      if (s.flags & H3_FLAG_VIDEO_CANVAS) {
+        h = canvas(y, s.grid_h, s.grid_h, s.grid_w);
+        w = canvas(x, s.grid_w, s.grid_h, s.grid_w);
+      } else {
+        h = static_cast<float>(y);
+        w = static_cast<float>(x);
+      }
     } else {  // H3_SEG_AUDIO
       const long long j = local / s.channels;
       const float c = static_cast<float>(local - j * s.channels);

@@ -128,7 +128,7 @@ h3_status h3_build_coords(const h3_segment* segs, int32_t nseg, const int32_t* d
       if (s.flags & ~H3_FLAG_TEXT_T_ONLY) return H3_ERR_INVALID_ARG;
       rows = s.count;
     } else if (s.kind == H3_SEG_VIDEO) {
-      if (s.flags != 0) return s.flags == H3_FLAG_VIDEO_CANVAS ? H3_ERR_UNSUPPORTED : H3_ERR_INVALID_ARG;
+      if (s.flags & ~H3_FLAG_VIDEO_CANVAS) return H3_ERR_INVALID_ARG;
       if (s.grid_h <= 0 || s.grid_w <= 0 || s.grid_h >= kExact || s.grid_w >= kExact)
         return H3_ERR_INVALID_ARG;
       rows = static_cast<long long>(s.count) * s.grid_h * s.grid_w;

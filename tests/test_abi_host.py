@@ -60,9 +60,9 @@ def test_build_coords_rejects_bad_tables():
                 0x1000) == h3.H3_ERR_INVALID_ARG
     assert _err(h3.h3_build_coords, [W.Segment(W.SEG_VIDEO, 3, 2, 2, 0, 0, 1 << 23, 3)], 0, 12,
                 0x1000) == h3.H3_ERR_INVALID_ARG
-    # reserved canvas mode is reported as unsupported
-    assert _err(h3.h3_build_coords, [W.Segment(W.SEG_VIDEO, 1, 2, 2, flags=4)], 0, 4,
-                0x1000) == h3.H3_ERR_UNSUPPORTED
+    # unknown video flag
+    assert _err(h3.h3_build_coords, [W.Segment(W.SEG_VIDEO, 1, 2, 2, flags=5)], 0, 4,
+                0x1000) == h3.H3_ERR_INVALID_ARG
     # too many segments, NULL output
     assert _err(h3.h3_build_coords, [W.text(1)] * 65, 0, 65, 0x1000) == h3.H3_ERR_INVALID_ARG
     assert _err(h3.h3_build_coords, [W.text(3)], 0, 3, 0) == h3.H3_ERR_INVALID_ARG

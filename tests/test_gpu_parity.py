@@ -235,3 +235,29 @@ def test_row_order_carries_no_position_on_gpu(h3):
     _sync_ok(h3)
     unshuffled = bf16_bits_to_f64(from_dev_bf16(o))
     assert np.abs(got - unshuffled[perm]).max() <= 2e-2
+
+
+# ------------------------------------------- normalised canvas, t-only text --
+
+def test_coords_canvas_bit_exact(h3):
+    segs = [W.text(7, flags=W.FLAG_TEXT_T_ONLY), W.video(2, 22, 40, flags=W.FLAG_VIDEO_CANVAS),
+            W.video(1, 44, 80, t_off_num=-300, flags=W.FLAG_VIDEO_CANVAS), W.video(3, 9, 16, flags=W.FLAG_VIDEO_CANVAS),
+            W.video(2, 5, 3, flags=W.FLAG_VIDEO_CANVAS), W.audio(11, 2)]
+    n = sum(s.rows for s in segs)
+    perm = W.fisher_yates(n, 123)
+    for p in (None, perm):
+        got = h3.build_coords(segs, n, _perm_dev(p)).cpu().numpy()
+        _sync_ok(h3)
+        _, want = ocoords.packed_values(segs, p)
+        assert got.tobytes() == want.tobytes()
+
+
+def test_pipeline_canvas_mode(h3):
+    # the pages' own positional scheme: text at (i, 0, 0), video on the canvas
+    segs = (W.text(128, flags=W.FLAG_TEXT_T_ONLY), W.video(5, 22, 40, flags=W.FLAG_VIDEO_CANVAS), W.audio(28, 2))
+    wl = W.Workload("small_canvas", 1, 8, 128, segs, shuffle=False)
+    q, k, v = W.qkv_bf16(wl)
+    o = h3.packed_mmrope_attention(segs, to_dev(q), to_dev(k), to_dev(v))
+    _sync_ok(h3)
+    ref, _ = opipe.packed_mmrope_attention(segs, None, q, k, v)
+    check_attention(bf16_bits_to_f64(from_dev_bf16(o)), ref, "canvas")
