@@ -162,6 +162,7 @@ def run_ours(args):
     nseg = len(wl.segments)
     L = _lib.load()
     rs = H * D
+    fused = args.fused_q_rope
 
     def call(status, what):
         if status != 0:
@@ -174,12 +175,21 @@ def run_ours(args):
                                coords.data_ptr(), s), "h3_build_coords")
         if evs is not None:
             evs[1].record(stream)
-        call(L.h3_mmrope_qk(dq.data_ptr(), dk.data_ptr(), dqr.data_ptr(), dkr.data_ptr(), coords.data_ptr(),
-                            N, H, rs, cfg, s), "h3_mmrope_qk")
+        if fused:
+            # K rotated by the rope kernel, Q rotated inside the attention kernel
+            call(L.h3_mmrope_qk(None, dk.data_ptr(), None, dkr.data_ptr(), coords.data_ptr(),
+                                N, H, rs, cfg, s), "h3_mmrope_qk")
+        else:
+            call(L.h3_mmrope_qk(dq.data_ptr(), dk.data_ptr(), dqr.data_ptr(), dkr.data_ptr(), coords.data_ptr(),
+                                N, H, rs, cfg, s), "h3_mmrope_qk")
         if evs is not None:
             evs[2].record(stream)
-        call(L.h3_packed_attention(dqr.data_ptr(), dkr.data_ptr(), dv.data_ptr(), do.data_ptr(), None, None,
-                                   None, 1, N, H, D, rs, 0.0, s), "h3_packed_attention")
+        if fused:
+            call(L.h3_packed_attention(dq.data_ptr(), dkr.data_ptr(), dv.data_ptr(), do.data_ptr(), None,
+                                       coords.data_ptr(), cfg, 1, N, H, D, rs, 0.0, s), "h3_packed_attention")
+        else:
+            call(L.h3_packed_attention(dqr.data_ptr(), dkr.data_ptr(), dv.data_ptr(), do.data_ptr(), None, None,
+                                       None, 1, N, H, D, rs, 0.0, s), "h3_packed_attention")
         if evs is not None:
             evs[3].record(stream)
 
@@ -251,14 +261,14 @@ def run_ours(args):
     pk, src = peaks()
     value = hdist.weak_scaling_throughput(flops, world, ms_per_step * 1e-3) / 1e12
     attn_tflops = flops / (attn_ms_max * 1e-3) / 1e12
-    rope_bytes = 4 * N * H * D * 2 + N * 12
+    rope_bytes = (2 if fused else 4) * N * H * D * 2 + N * 12
     rope_gbs = rope_bytes / (rope_ms * 1e-3) / 1e9
     traffic = profiled_traffic(wl)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16)",
-        "config": config_dict(wl, world),
+        "config": dict(config_dict(wl, world), rope_fused_into_attention=("Q" if fused else "none")),
         "pct_bf16_peak": round(100 * value / world / pk["bf16_tflops_sustained"], 2),
         "kernels_ms": {"h3_build_coords": round(coords_ms, 4), "h3_mmrope_qk": round(rope_ms, 4),
                        "h3_packed_attention": round(attn_ms, 4)},
@@ -370,6 +380,8 @@ def main():
     ap.add_argument("--config", type=int, default=2, help="workload index (default 2: 28,196 rows)")
     ap.add_argument("--video-frames", type=int, default=0,
                     help="resize the worked-example layout to this many latent frames (profiling cases)")
+    ap.add_argument("--fused-q-rope", action="store_true",
+                    help="rotate only K in h3_mmrope_qk and Q inside h3_packed_attention")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=128, help="query rows of the timed oracle sample")
     ap.add_argument("--ref-rows", type=int, default=16, help="query rows per reference-arm step")

@@ -157,7 +157,9 @@ h3_status h3_build_coords(const h3_segment* segs, int32_t nseg, const int32_t* d
  *
  *   d_q, d_k          device bf16 inputs, layout above (batch folded into rows)
  *   d_q_out, d_k_out  device bf16 outputs, same layout and stride; may equal
- *                     the inputs (in place); must not partially overlap them
+ *                     the inputs (in place); must not partially overlap them.
+ *                     d_q and d_q_out may both be NULL: then only K is rotated
+ *                     (the partner of h3_packed_attention's fused Q rotation)
  *   d_coords          device float[n_rows][3] from h3_build_coords
  *   n_rows, n_heads   rows and heads; row_stride in elements
  *   cfg               host rotary configuration
@@ -182,16 +184,21 @@ h3_status h3_mmrope_qk(const void* d_q, const void* d_k, void* d_q_out, void* d_
  *   d_o             device bf16 output, same layout and row_stride
  *   d_lse           device float[batch][n_heads][n_rows] natural-log row
  *                   log-sum-exp of the scaled logits, or NULL
- *   d_coords, cfg   must be NULL: rotation fused into the tile load is not
- *                   available in this version (H3_ERR_UNSUPPORTED)
+ *   d_coords, cfg   NULL: Q and K arrive rotated.  Non-NULL (device float
+ *                   [batch][n_rows][3] from h3_build_coords, host cfg): Q arrives
+ *                   UNROTATED and each CTA rotates its Q tiles in shared memory
+ *                   as they are loaded, with exactly the arithmetic of
+ *                   h3_mmrope_qk (so O is identical to rotating first); K must
+ *                   already be rotated (h3_mmrope_qk with d_q = NULL).  Rotating K
+ *                   here would repeat the work in every query-tile CTA of a head.
  *   softmax_scale   > 0, or <= 0 for 1/sqrt(head_dim)
  * Arithmetic: bf16 tensor-core products with fp32 accumulation (tcgen05),
  * fp32 online softmax, P rounded to bf16 for the P.V product, O rounded to
  * bf16.  All waits inside the kernel are bounded; on expiry the kernel stops
  * and h3_check_device_error returns H3_ERR_TIMEOUT.
  * Errors: H3_ERR_INVALID_ARG (NULL pointers with n_rows > 0, n_rows >= 2^31,
- * batch or n_heads < 1, bad stride); H3_ERR_UNSUPPORTED (head_dim != 128,
- * misaligned pointer or stride, d_coords != NULL).
+ * batch or n_heads < 1, bad stride, bad cfg with d_coords); H3_ERR_UNSUPPORTED
+ * (head_dim != 128, misaligned pointer or stride).
  */
 h3_status h3_packed_attention(const void* d_q, const void* d_k, const void* d_v, void* d_o,
                               float* d_lse, const float* d_coords, const h3_rope_cfg* cfg,

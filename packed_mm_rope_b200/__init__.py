@@ -58,24 +58,36 @@ def build_coords(segments, n_rows: int, perm=None, out=None, stream=None):
 
 def mmrope_qk(q, k, coords, q_out=None, k_out=None, theta=10000.0, sections=(32, 48, 48), pair_layout=0,
               stream=None):
-    """Rotate Q and K; returns (q_out, k_out).  Pass q_out=q, k_out=k for in place."""
+    """Rotate Q and K; returns (q_out, k_out).  Pass q_out=q, k_out=k for in place.
+
+    q=None rotates K only (returns (None, k_out)).
+    """
     import torch
-    b, n, h, rs = _row_layout(q)
-    if _row_layout(k) != (b, n, h, rs):
+    b, n, h, rs = _row_layout(k)
+    if q is not None and _row_layout(q) != (b, n, h, rs):
         raise ValueError("q and k layouts differ")
-    q_out = torch.empty_like(q) if q_out is None else q_out
+    if q is not None:
+        q_out = torch.empty_like(q) if q_out is None else q_out
+        if _row_layout(q_out) != (b, n, h, rs):
+            raise ValueError("outputs must share the inputs' layout")
     k_out = torch.empty_like(k) if k_out is None else k_out
-    if _row_layout(q_out) != (b, n, h, rs) or _row_layout(k_out) != (b, n, h, rs):
+    if _row_layout(k_out) != (b, n, h, rs):
         raise ValueError("outputs must share the inputs' layout")
     if coords.dtype != torch.float32 or coords.numel() != 3 * b * n or not coords.is_contiguous():
         raise ValueError("coords must be contiguous fp32 [rows, 3]")
-    h3_mmrope_qk(q.data_ptr(), k.data_ptr(), q_out.data_ptr(), k_out.data_ptr(), coords.data_ptr(), b * n, h,
+    h3_mmrope_qk(q.data_ptr() if q is not None else 0, k.data_ptr(),
+                 q_out.data_ptr() if q is not None else 0, k_out.data_ptr(), coords.data_ptr(), b * n, h,
                  rs, rope_cfg(theta, 128, sections, pair_layout), _stream(stream))
-    return q_out, k_out
+    return (q_out if q is not None else None), k_out
 
 
-def packed_attention(q, k, v, out=None, lse=None, softmax_scale: float = 0.0, stream=None):
-    """O = softmax(Q K^T * scale) V over all packed rows, per head."""
+def packed_attention(q, k, v, out=None, lse=None, softmax_scale: float = 0.0, stream=None, coords=None,
+                     theta=10000.0, sections=(32, 48, 48), pair_layout=0):
+    """O = softmax(Q K^T * scale) V over all packed rows, per head.
+
+    With ``coords`` (fp32 [rows, 3]) Q is passed UNROTATED and rotated inside
+    the kernel as its tiles are loaded; K must already be rotated.
+    """
     import torch
     lay = _row_layout(q)
     if _row_layout(k) != lay or _row_layout(v) != lay:
@@ -89,19 +101,30 @@ def packed_attention(q, k, v, out=None, lse=None, softmax_scale: float = 0.0, st
         if lse.dtype != torch.float32 or lse.numel() != b * h * n or not lse.is_contiguous():
             raise ValueError("lse must be contiguous fp32 [B, H, N]")
         lp = lse.data_ptr()
+    cp, cfg = 0, None
+    if coords is not None:
+        if coords.dtype != torch.float32 or coords.numel() != 3 * b * n or not coords.is_contiguous():
+            raise ValueError("coords must be contiguous fp32 [rows, 3]")
+        cp, cfg = coords.data_ptr(), rope_cfg(theta, 128, sections, pair_layout)
     h3_packed_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lp, b, n, h, rs,
-                        softmax_scale, stream=_stream(stream))
+                        softmax_scale, d_coords=cp, cfg=cfg, stream=_stream(stream))
     return out
 
 
 def packed_mmrope_attention(segments, q, k, v, perm=None, theta=10000.0, sections=(32, 48, 48),
-                            pair_layout=0, out=None, lse=None, softmax_scale: float = 0.0, stream=None):
+                            pair_layout=0, out=None, lse=None, softmax_scale: float = 0.0, stream=None,
+                            fused_q_rope: bool = False):
     """The whole path on one packed sequence: coords -> rotate Q, K -> attention.
 
     q, k, v: [N, H, 128] bf16 on the GPU (unrotated).  Returns O [N, H, 128].
+    fused_q_rope: rotate only K beforehand and Q inside the attention kernel.
     """
-    import torch
     n = q.shape[-3]
     coords = build_coords(segments, n, perm, stream=stream)
+    if fused_q_rope:
+        _, kr = mmrope_qk(None, k, coords, theta=theta, sections=sections, pair_layout=pair_layout,
+                          stream=stream)
+        return packed_attention(q, kr, v, out=out, lse=lse, softmax_scale=softmax_scale, stream=stream,
+                                coords=coords, theta=theta, sections=sections, pair_layout=pair_layout)
     qr, kr = mmrope_qk(q, k, coords, theta=theta, sections=sections, pair_layout=pair_layout, stream=stream)
     return packed_attention(qr, kr, v, out=out, lse=lse, softmax_scale=softmax_scale, stream=stream)

@@ -47,6 +47,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "rope.cuh"
 
 namespace h3 {
 namespace attn {
@@ -67,8 +68,9 @@ constexpr uint32_t SMEM_Q = 0;
 constexpr uint32_t SMEM_KV = 2 * TILE_BYTES;
 constexpr uint32_t SMEM_BAR = SMEM_KV + KV_STAGES * TILE_BYTES;
 // barriers: q_full[2], kv_full[S], kv_empty[S], s_full[2], p_full[2][2] (halves),
-//           pva_done[2] (first half of PV landed), o_full[2], mma_done
-constexpr int NUM_BARS = 2 + 2 * KV_STAGES + 2 + 4 + 2 + 2 + 1;
+//           pva_done[2] (first half of PV landed), o_full[2], mma_done,
+//           q_ready[2] (Q tile rotated in place, fused RoPE only)
+constexpr int NUM_BARS = 2 + 2 * KV_STAGES + 2 + 4 + 2 + 2 + 1 + 2;
 constexpr uint32_t SMEM_MISC = SMEM_BAR + NUM_BARS * 8;   // tmem base, abort flag
 constexpr uint32_t SMEM_BYTES = SMEM_MISC + 16 + 1024;    // + alignment slack
 
@@ -150,6 +152,10 @@ struct Params {
   float* lse;                     // [B][H][N] or null
   unsigned long long wait_limit_ns;
   unsigned long long drain_limit_ns;
+  // fused RoPE on Q (coords == null: Q arrives rotated)
+  const float* coords;            // [B][N][3]
+  int rope_layout;                // 0 adjacent pairs, 1 half-split
+  RopeTable rope;
 };
 
 // 2^(x*sl2 - m) for 64 logits: bf16 pairs and their sum.  Two logits per
@@ -207,6 +213,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   auto bar_pva_done = [&](int i) { return bar0 + 8u * (8 + 2 * KV_STAGES + i); };
   auto bar_o_full = [&](int i) { return bar0 + 8u * (10 + 2 * KV_STAGES + i); };
   const uint32_t bar_mma_done = bar0 + 8u * (12 + 2 * KV_STAGES);
+  auto bar_q_ready = [&](int i) { return bar0 + 8u * (13 + 2 * KV_STAGES + i); };
+  const bool fused_rope = p.coords != nullptr;
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gbase + SMEM_MISC);
   volatile uint32_t* const abort_flag = reinterpret_cast<volatile uint32_t*>(gbase + SMEM_MISC + 4);
 
@@ -232,6 +240,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       mbar_init(bar_kv_empty(s), 1);
     }
     mbar_init(bar_mma_done, 1);
+    mbar_init(bar_q_ready(0), 128);
+    mbar_init(bar_q_ready(1), 128);
     *abort_flag = 0u;
     mbar_fence_init();
   }
@@ -318,13 +328,15 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         issue_pv(i, vs, 1, true);
         return true;
       };
-      bool ok = mma_wait(bar_q_full(0), 0, abort_flag, limit) &&
+      // with fused RoPE the softmax warpgroups rotate Q in place first
+      auto bar_q = [&](int i) { return fused_rope ? bar_q_ready(i) : bar_q_full(i); };
+      bool ok = mma_wait(bar_q(0), 0, abort_flag, limit) &&
                 mma_wait(bar_kv_full(0), 0, abort_flag, limit);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
         tc_commit(bar_s_full(0));
-        ok = mma_wait(bar_q_full(1), 0, abort_flag, limit);
+        ok = mma_wait(bar_q(1), 0, abort_flag, limit);
       }
       if (ok) {
         tc_fence_after();
@@ -404,6 +416,45 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tc_fence_before();
       mbar_arrive(bar_p_full(wg, half));
     };
+
+    // Fused RoPE: rotate this warpgroup's Q tile in shared memory, one thread
+    // per row, with the rope kernel's arithmetic (rope_cos_sin, rot2), then
+    // make the generic-proxy writes visible to the tensor core (async proxy).
+    if (fused_rope) {
+      if (!warp_wait(bar_q_full(wg), 0, abort_flag, limit)) ok = false;
+      const int row = q_row0 + wg * BM + row_in_tile;
+      if (ok && row < p.n_rows) {
+        const float* crd = p.coords + (static_cast<long long>(batch) * p.n_rows + row) * 3;
+        const float c3[3] = {crd[0], crd[1], crd[2]};
+        uint8_t* qrow = gbase + SMEM_Q + wg * TILE_BYTES + row_in_tile * 128;
+        const int sw = row_in_tile & 7;           // 128-byte swizzle of this row
+        auto chunk = [&](int c) {                 // logical 16-byte chunk c of 16
+          return reinterpret_cast<uint4*>(qrow + (c >> 3) * HALF_BYTES + (((c & 7) ^ sw) << 4));
+        };
+        if (p.rope_layout == 0) {
+#pragma unroll 1
+          for (int c = 0; c < 16; ++c) {
+            float2 cs[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) cs[m] = rope_cos_sin(p.rope, c3, 4 * c + m);
+            *chunk(c) = rotate_adjacent(*chunk(c), cs);
+          }
+        } else {
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            float2 cs[8];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) cs[m] = rope_cos_sin(p.rope, c3, 8 * c + m);
+            uint4 a = *chunk(c), b = *chunk(c + 8);
+            rotate_half(a, b, cs);
+            *chunk(c) = a;
+            *chunk(c + 8) = b;
+          }
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(bar_q_ready(wg));
+    }
 
     for (int j = 0; j < nkv; ++j) {
       if (!warp_wait(bar_s_full(wg), j & 1, abort_flag, limit)) { ok = false; break; }

@@ -167,7 +167,8 @@ h3_status h3_mmrope_qk(const void* d_q, const void* d_k, void* d_q_out, void* d_
   if (cfg->head_dim != 128) return H3_ERR_UNSUPPORTED;
   if (row_stride < static_cast<int64_t>(n_heads) * 128) return H3_ERR_INVALID_ARG;
   if (n_rows == 0) return H3_OK;
-  if (!d_q || !d_k || !d_q_out || !d_k_out || !d_coords) return H3_ERR_INVALID_ARG;
+  if ((d_q == nullptr) != (d_q_out == nullptr)) return H3_ERR_INVALID_ARG;   // both or neither
+  if (!d_k || !d_k_out || !d_coords) return H3_ERR_INVALID_ARG;
   if (row_stride % 8 != 0 || !aligned16(d_q) || !aligned16(d_k) || !aligned16(d_q_out) ||
       !aligned16(d_k_out))
     return H3_ERR_UNSUPPORTED;
@@ -194,10 +195,12 @@ h3_status h3_packed_attention(const void* d_q, const void* d_k, const void* d_v,
                               const float* d_coords, const h3_rope_cfg* cfg, int32_t batch, int64_t n_rows,
                               int32_t n_heads, int32_t head_dim, int64_t row_stride, float softmax_scale,
                               void* stream) {
-  (void)cfg;
   if (batch < 1 || n_heads < 1 || n_rows < 0 || n_rows >= (1ll << 31)) return H3_ERR_INVALID_ARG;
   if (head_dim != 128) return H3_ERR_UNSUPPORTED;
-  if (d_coords != nullptr) return H3_ERR_UNSUPPORTED;
+  if (d_coords != nullptr) {
+    if (!valid_rope_cfg(cfg)) return H3_ERR_INVALID_ARG;
+    if (cfg->head_dim != 128) return H3_ERR_UNSUPPORTED;
+  }
   if (row_stride < static_cast<int64_t>(n_heads) * 128) return H3_ERR_INVALID_ARG;
   if (batch > 65535 || n_heads > 65535) return H3_ERR_INVALID_ARG;
   if (!std::isfinite(softmax_scale)) return H3_ERR_INVALID_ARG;
@@ -230,6 +233,10 @@ h3_status h3_packed_attention(const void* d_q, const void* d_k, const void* d_v,
   p.lse = d_lse;
   p.wait_limit_ns = g_wait_limit_ns;
   p.drain_limit_ns = kDrainLimitNs;
+  p.coords = d_coords;
+  p.rope_layout = d_coords ? cfg->pair_layout : 0;
+  if (d_coords) p.rope = make_rope_table(cfg);
+  else std::memset(&p.rope, 0, sizeof(p.rope));
   const dim3 grid(static_cast<unsigned>((n_rows + 2 * h3::attn::BM - 1) / (2 * h3::attn::BM)),
                   static_cast<unsigned>(n_heads), static_cast<unsigned>(batch));
   h3::attn::attention_kernel<<<grid, h3::attn::THREADS, h3::attn::SMEM_BYTES, as_stream(stream)>>>(tq, tk, tv,

@@ -26,9 +26,22 @@ constexpr int ROPE_THREADS = 256;
 constexpr int ROPE_ROWS = 8;      // rows per block iteration
 constexpr int ROPE_UNROLL = 4;    // independent 16-byte chunks in flight per thread
 
+// (cos, sin) of pair p for a row with coordinates crd[0..2]: fp64 angle =
+// fp64(coordinate) x fp64 inverse frequency, fp64 sincos, each rounded to fp32.
+// Shared by the rope kernel and the attention kernel's fused Q rotation, so
+// both produce identical rotated values.
+__device__ __forceinline__ float2 rope_cos_sin(const RopeTable& tab, const float* crd, int p) {
+  const double a = static_cast<double>(crd[tab.axis[p]]) * tab.inv_freq[p];
+  double sn, cn;
+  sincos(a, &sn, &cn);
+  return make_float2(static_cast<float>(cn), static_cast<float>(sn));
+}
+
+// (x0, x1) -> (x0 c - x1 s, x0 s + x1 c) with every rounding explicit (no
+// compiler-chosen contraction), so the result does not depend on the caller.
 __device__ __forceinline__ void rot2(float x0, float x1, float2 cs, float& y0, float& y1) {
-  y0 = x0 * cs.x - x1 * cs.y;
-  y1 = x0 * cs.y + x1 * cs.x;
+  y0 = __fmaf_rn(x0, cs.x, -__fmul_rn(x1, cs.y));
+  y1 = __fmaf_rn(x0, cs.y, __fmul_rn(x1, cs.x));
 }
 
 // Rotate 4 adjacent pairs held in one 16-byte chunk (8 bf16).
@@ -62,6 +75,7 @@ __device__ __forceinline__ void rotate_half(uint4& a, uint4& b, const float2* cs
   b = make_uint4(wb[0], wb[1], wb[2], wb[3]);
 }
 
+// q / qo may both be null: then only K is rotated.
 // LAYOUT 0: pair p = dims (2p, 2p+1); one work item = one 16-byte chunk.
 // LAYOUT 1: pair p = dims (p, p+64);  one work item = chunks c and c+8 of a head.
 template <int LAYOUT>
@@ -79,10 +93,7 @@ __global__ void __launch_bounds__(ROPE_THREADS) rope_kernel(
     __syncthreads();   // previous block's readers are done with cs
     for (int i = threadIdx.x; i < nr * 64; i += ROPE_THREADS) {
       const int r = i >> 6, p = i & 63;
-      const double a = static_cast<double>(coords[3 * (r0 + r) + tab.axis[p]]) * tab.inv_freq[p];
-      double sn, cn;
-      sincos(a, &sn, &cn);
-      cs[r][p] = make_float2(static_cast<float>(cn), static_cast<float>(sn));
+      cs[r][p] = rope_cos_sin(tab, coords + 3 * (r0 + r), p);
     }
     __syncthreads();
 
@@ -103,10 +114,10 @@ __global__ void __launch_bounds__(ROPE_THREADS) rope_kernel(
           row[u] = r;
           off[u] = (r0 + r) * stride16 + head * 16 + sub;
           pair0[u] = LAYOUT == 0 ? 4 * sub : 8 * sub;
-          qa[u] = __ldcs(q + off[u]);
+          if (q != nullptr) qa[u] = __ldcs(q + off[u]);
           ka[u] = __ldcs(k + off[u]);
           if (LAYOUT == 1) {
-            qb[u] = __ldcs(q + off[u] + 8);
+            if (q != nullptr) qb[u] = __ldcs(q + off[u] + 8);
             kb[u] = __ldcs(k + off[u] + 8);
           }
         }
@@ -116,13 +127,15 @@ __global__ void __launch_bounds__(ROPE_THREADS) rope_kernel(
         if (off[u] < 0) continue;
         const float2* c = &cs[row[u]][pair0[u]];
         if (LAYOUT == 0) {
-          __stcs(qo + off[u], rotate_adjacent(qa[u], c));
+          if (q != nullptr) __stcs(qo + off[u], rotate_adjacent(qa[u], c));
           __stcs(ko + off[u], rotate_adjacent(ka[u], c));
         } else {
-          rotate_half(qa[u], qb[u], c);
+          if (q != nullptr) {
+            rotate_half(qa[u], qb[u], c);
+            __stcs(qo + off[u], qa[u]);
+            __stcs(qo + off[u] + 8, qb[u]);
+          }
           rotate_half(ka[u], kb[u], c);
-          __stcs(qo + off[u], qa[u]);
-          __stcs(qo + off[u] + 8, qb[u]);
           __stcs(ko + off[u], ka[u]);
           __stcs(ko + off[u] + 8, kb[u]);
         }

@@ -88,7 +88,8 @@ def test_rope_rejects_bad_config_and_layout():
     assert _err(h3.h3_mmrope_qk, P, P, P, P, P, 4, 2, 128, h3.rope_cfg()) == h3.H3_ERR_INVALID_ARG
     assert _err(h3.h3_mmrope_qk, P, P, P, P, P, 4, 1, 132, h3.rope_cfg()) == h3.H3_ERR_UNSUPPORTED
     assert _err(h3.h3_mmrope_qk, P + 8, P, P, P, P, 4, 1, 128, h3.rope_cfg()) == h3.H3_ERR_UNSUPPORTED
-    assert _err(h3.h3_mmrope_qk, 0, P, P, P, P, 4, 1, 128, h3.rope_cfg()) == h3.H3_ERR_INVALID_ARG
+    assert _err(h3.h3_mmrope_qk, 0, P, P, P, P, 4, 1, 128, h3.rope_cfg()) == h3.H3_ERR_INVALID_ARG   # q out without q
+    assert _err(h3.h3_mmrope_qk, 0, 0, 0, P, P, 4, 1, 128, h3.rope_cfg()) == h3.H3_ERR_INVALID_ARG   # no k
 
 
 def test_attention_rejects_bad_arguments():
@@ -102,5 +103,7 @@ def test_attention_rejects_bad_arguments():
     assert _err(A, P, P, P, P, 0, 1, 10, 1, 132) == h3.H3_ERR_UNSUPPORTED
     assert _err(A, P, P, P + 4, P, 0, 1, 10, 1, 128) == h3.H3_ERR_UNSUPPORTED
     assert _err(A, P, P, 0, P, 0, 1, 10, 1, 128) == h3.H3_ERR_INVALID_ARG
-    assert _err(A, P, P, P, P, 0, 1, 10, 1, 128, d_coords=P) == h3.H3_ERR_UNSUPPORTED
+    assert _err(A, P, P, P, P, 0, 1, 10, 1, 128, d_coords=P) == h3.H3_ERR_INVALID_ARG     # no cfg
+    assert _err(A, P, P, P, P, 0, 1, 10, 1, 128, d_coords=P,
+                cfg=h3.rope_cfg(sections=(32, 48, 40))) == h3.H3_ERR_INVALID_ARG
     assert _err(A, P, P, P, P, 0, 1, 10, 1, 128, softmax_scale=float("nan")) == h3.H3_ERR_INVALID_ARG

@@ -261,3 +261,48 @@ def test_pipeline_canvas_mode(h3):
     _sync_ok(h3)
     ref, _ = opipe.packed_mmrope_attention(segs, None, q, k, v)
     check_attention(bf16_bits_to_f64(from_dev_bf16(o)), ref, "canvas")
+
+
+# -------------------------------------------------- fused RoPE on Q (a5) --
+
+@pytest.mark.parametrize("cfg,layout", [(0, 0), (1, 0), (1, 1)])
+def test_fused_q_rope_is_identical_to_rotating_first(h3, cfg, layout):
+    wl = W.workload(cfg)
+    perm = W.permutation(wl)
+    q, k, v = W.qkv_bf16(wl)
+    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+    args = dict(perm=_perm_dev(perm), theta=wl.theta, sections=wl.sections, pair_layout=layout)
+    o_sep = h3.packed_mmrope_attention(wl.segments, dq, dk, dv, **args)
+    o_fus = h3.packed_mmrope_attention(wl.segments, dq, dk, dv, fused_q_rope=True, **args)
+    _sync_ok(h3)
+    # same rotation arithmetic, same MMAs: bit-identical outputs
+    assert torch.equal(o_sep, o_fus)
+    ref, _ = opipe.packed_mmrope_attention(wl.segments, perm, q, k, v, wl.theta, wl.sections, pair_layout=layout)
+    check_attention(bf16_bits_to_f64(from_dev_bf16(o_fus)), ref, f"fused {wl.name}")
+
+
+def test_rope_k_only_leaves_q_alone(h3):
+    wl = W.workload(0)
+    perm = W.permutation(wl)
+    q, k, _ = W.qkv_bf16(wl)
+    coords = h3.build_coords(wl.segments, wl.n_rows, _perm_dev(perm))
+    dq, dk = to_dev(q), to_dev(k)
+    q_both, k_both = h3.mmrope_qk(dq, dk, coords)
+    none, k_only = h3.mmrope_qk(None, dk, coords)
+    _sync_ok(h3)
+    assert none is None and torch.equal(k_only, k_both)
+    assert torch.equal(dq, to_dev(q))
+
+
+def test_fused_q_rope_ragged_batch(h3):
+    B, N, H = 2, 300, 3
+    segs = [W.text(20), W.video(2, 10, 12, flags=W.FLAG_VIDEO_CANVAS), W.audio(20, 2)]
+    assert sum(s.rows for s in segs) == N
+    q, k, v = (W.normal_bf16(400 + i, 0, (B, N, H, 128)) for i in range(3))
+    coords = torch.cat([h3.build_coords(segs, N) for _ in range(B)])      # [B*N, 3]
+    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+    qr, kr = h3.mmrope_qk(dq, dk, coords)
+    o_sep = h3.packed_attention(qr, kr, dv)
+    o_fus = h3.packed_attention(dq, kr, dv, coords=coords)
+    _sync_ok(h3)
+    assert torch.equal(o_sep, o_fus)
