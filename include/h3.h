@@ -206,6 +206,46 @@ h3_status h3_packed_attention(const void* d_q, const void* d_k, const void* d_v,
                               int64_t row_stride, float softmax_scale, void* stream);
 
 /*
+ * Device workspace, in bytes, that h3_packed_mmrope_attention_host needs for
+ * n_rows x n_heads (Q, K, V, O copies, coordinates and the permutation,
+ * each 256-byte aligned).  Returns 0 for invalid sizes.
+ */
+uint64_t h3_host_workspace_bytes(int64_t n_rows, int32_t n_heads);
+
+/*
+ * h3_packed_mmrope_attention_host -- the whole path (coords, MM-RoPE on Q and
+ * K, full attention) for one packed sequence whose Q, K, V and O live in HOST
+ * memory.  Same operation and arithmetic as h3_build_coords + h3_mmrope_qk +
+ * h3_packed_attention (same passages), pipelined over chunks of heads: while
+ * chunk c is rotated and attended on the GPU, chunk c+1 is copied in and
+ * chunk c-1's O is copied out, on two internal copy streams ordered by events.
+ *
+ *   segs, nseg        host segment table (as h3_build_coords)
+ *   h_perm            host int32[n_rows] row permutation, or NULL
+ *   h_q, h_k, h_v     host bf16 [n_rows][n_heads][128], contiguous; pinned
+ *                     memory (cudaHostAlloc / cudaHostRegister) for the copies
+ *                     to overlap, pageable memory works but serialises
+ *   h_o               host bf16 output, same layout
+ *   d_work            device workspace of h3_host_workspace_bytes() bytes,
+ *                     256-byte aligned, owned by the caller; contents undefined
+ *                     after the call
+ *   heads_per_chunk   0 = chosen by the library (chunks whose CTA count fills
+ *                     whole waves of SMs), else 1..n_heads
+ *   cfg               host rotary configuration
+ *   stream            work starts after everything already queued on `stream`;
+ *                     the call returns once all work is queued, and `stream`
+ *                     is ordered after the last copy out: synchronise `stream`
+ *                     to wait for h_o.  Host buffers must stay valid until then.
+ * Errors: as the three calls it composes; H3_ERR_INVALID_ARG for a NULL or
+ * misaligned workspace; H3_ERR_CUDA if an internal stream or event cannot be
+ * created (they are created once per device and kept until process exit).
+ */
+h3_status h3_packed_mmrope_attention_host(const h3_segment* segs, int32_t nseg, const int32_t* h_perm,
+                                          const void* h_q, const void* h_k, const void* h_v, void* h_o,
+                                          void* d_work, int64_t n_rows, int32_t n_heads,
+                                          int32_t heads_per_chunk, const h3_rope_cfg* cfg, void* stream);
+
+/*
  * Synchronise `stream`, then read and clear this device's error word.
  * Returns H3_OK, H3_ERR_TIMEOUT, H3_ERR_DEVICE_INPUT or H3_ERR_CUDA.
  */

@@ -16,7 +16,8 @@ from __future__ import annotations
 from . import _lib
 from ._lib import (H3Error, H3_OK, H3_ERR_INVALID_ARG, H3_ERR_UNSUPPORTED, H3_ERR_CUDA,  # noqa: F401
                    H3_ERR_TIMEOUT, H3_ERR_DEVICE_INPUT, h3_build_coords, h3_check_device_error,
-                   h3_mmrope_qk, h3_packed_attention, h3_set_wait_limit_ns, rope_cfg, status_str)
+                   h3_host_workspace_bytes, h3_mmrope_qk, h3_packed_attention, h3_packed_mmrope_attention_host,
+                   h3_set_wait_limit_ns, rope_cfg, status_str)
 
 LIB = _lib.load()
 
@@ -128,3 +129,40 @@ def packed_mmrope_attention(segments, q, k, v, perm=None, theta=10000.0, section
                                 coords=coords, theta=theta, sections=sections, pair_layout=pair_layout)
     qr, kr = mmrope_qk(q, k, coords, theta=theta, sections=sections, pair_layout=pair_layout, stream=stream)
     return packed_attention(qr, kr, v, out=out, lse=lse, softmax_scale=softmax_scale, stream=stream)
+
+
+def host_workspace(n_rows: int, n_heads: int, device=None):
+    """A device workspace (uint8 tensor) for packed_mmrope_attention_host."""
+    import torch
+    nbytes = h3_host_workspace_bytes(n_rows, n_heads)
+    if nbytes == 0:
+        raise ValueError("invalid sizes")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
+
+
+def packed_mmrope_attention_host(segments, q, k, v, out=None, perm=None, workspace=None, theta=10000.0,
+                                 sections=(32, 48, 48), pair_layout=0, heads_per_chunk: int = 0, stream=None):
+    """The whole path from and to HOST memory, copies overlapped with compute.
+
+    q, k, v: CPU bf16 [N, H, 128] contiguous tensors (pin them for overlap);
+    perm: CPU int32 [N] or None.  Returns the CPU output (``out`` if given).
+    Work is queued on ``stream``; synchronise it before reading the output.
+    """
+    import torch
+    for t in (q, k, v):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != q.shape:
+            raise ValueError("q, k, v must be contiguous CPU bf16 tensors of one shape")
+    n, h = q.shape[-3], q.shape[-2]
+    if q.dim() != 3 or q.shape[-1] != 128:
+        raise ValueError("expected [N, H, 128]")
+    if out is None:
+        out = torch.empty_like(q, pin_memory=q.is_pinned())
+    if perm is not None and (perm.dtype != torch.int32 or perm.is_cuda or perm.numel() != n):
+        raise ValueError("perm must be a CPU int32 tensor of N entries")
+    if workspace is None:
+        workspace = host_workspace(n, h)
+    h3_packed_mmrope_attention_host(segments, perm.data_ptr() if perm is not None else 0, q.data_ptr(),
+                                    k.data_ptr(), v.data_ptr(), out.data_ptr(), workspace.data_ptr(), n, h,
+                                    rope_cfg(theta, 128, sections, pair_layout), heads_per_chunk,
+                                    _stream(stream))
+    return out

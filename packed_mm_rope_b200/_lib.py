@@ -18,7 +18,8 @@ H3_FLAG_TEXT_T_ONLY, H3_FLAG_AUDIO_CHANNEL_H, H3_FLAG_VIDEO_CANVAS = 1, 2, 4
 H3_MAX_SEGMENTS = 64
 
 EXPORTED = ("h3_status_str", "h3_version", "h3_build_coords", "h3_mmrope_qk",
-            "h3_packed_attention", "h3_check_device_error", "h3_set_wait_limit_ns")
+            "h3_packed_attention", "h3_check_device_error", "h3_set_wait_limit_ns",
+            "h3_host_workspace_bytes", "h3_packed_mmrope_attention_host")
 
 
 class h3_segment(ctypes.Structure):
@@ -65,6 +66,11 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.h3_check_device_error.argtypes = [P]
     lib.h3_set_wait_limit_ns.restype = I32
     lib.h3_set_wait_limit_ns.argtypes = [U64]
+    lib.h3_host_workspace_bytes.restype = U64
+    lib.h3_host_workspace_bytes.argtypes = [I64, I32]
+    lib.h3_packed_mmrope_attention_host.restype = I32
+    lib.h3_packed_mmrope_attention_host.argtypes = [ctypes.POINTER(h3_segment), I32, P, P, P, P, P, P, I64, I32,
+                                                    I32, ctypes.POINTER(h3_rope_cfg), P]
     _lib = lib
     return lib
 
@@ -112,6 +118,20 @@ def h3_packed_attention(d_q: int, d_k: int, d_v: int, d_o: int, d_lse: int, batc
                                       d_coords or None, ctypes.byref(cfg) if cfg is not None else None,
                                       batch, n_rows, n_heads, head_dim, row_stride, softmax_scale,
                                       stream or None), "h3_packed_attention")
+
+
+def h3_host_workspace_bytes(n_rows: int, n_heads: int) -> int:
+    return int(load().h3_host_workspace_bytes(n_rows, n_heads))
+
+
+def h3_packed_mmrope_attention_host(segments, h_perm: int, h_q: int, h_k: int, h_v: int, h_o: int, d_work: int,
+                                    n_rows: int, n_heads: int, cfg: h3_rope_cfg, heads_per_chunk: int = 0,
+                                    stream: int = 0) -> None:
+    arr = segment_array(segments)
+    _check(load().h3_packed_mmrope_attention_host(arr, len(segments), h_perm or None, h_q or None, h_k or None,
+                                                  h_v or None, h_o or None, d_work or None, n_rows, n_heads,
+                                                  heads_per_chunk, ctypes.byref(cfg), stream or None),
+           "h3_packed_mmrope_attention_host")
 
 
 def h3_check_device_error(stream: int = 0) -> int:

@@ -171,7 +171,7 @@ __device__ __forceinline__ void exp_half(const float (&x)[64], float sl2, float 
   for (int c = 0; c < 32; ++c) {
     const float2 y = __ffma2_rn(make_float2(x[2 * c], x[2 * c + 1]), c2, mm);
     float p0, p1;
-    if (EXP2_FMA_EVERY > 0 && (c % EXP2_FMA_EVERY) == EXP2_FMA_EVERY - 1) {
+    if (EXP2_FMA_EVERY > 0 && (c % (EXP2_FMA_EVERY > 0 ? EXP2_FMA_EVERY : 1)) == EXP2_FMA_EVERY - 1) {
       const float2 e = exp2_fma2(y);
       p0 = e.x;
       p1 = e.y;

@@ -244,6 +244,136 @@ h3_status h3_packed_attention(const void* d_q, const void* d_k, const void* d_v,
   return cudaGetLastError() == cudaSuccess ? H3_OK : H3_ERR_CUDA;
 }
 
+uint64_t h3_host_workspace_bytes(int64_t n_rows, int32_t n_heads) {
+  if (n_rows <= 0 || n_heads < 1 || n_rows >= (1ll << 31)) return 0;
+  auto up = [](uint64_t b) { return (b + 255u) & ~uint64_t(255u); };
+  const uint64_t t = static_cast<uint64_t>(n_rows) * n_heads * 128u * 2u;
+  return 4 * up(t) + up(static_cast<uint64_t>(n_rows) * 12u) + up(static_cast<uint64_t>(n_rows) * 4u);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Streams and events of the host-buffer pipeline: created once per device,
+// kept for the life of the process.
+struct HostPipe {
+  std::mutex enqueue;             // one caller at a time enqueues on a device
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  static constexpr int kEvents = 3 * 64 + 2;
+  cudaEvent_t ev[kEvents] = {};
+  bool ok = false;
+};
+
+HostPipe* host_pipe() {
+  static std::mutex mu;
+  static HostPipe pipes[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  HostPipe& hp = pipes[dev];
+  if (!hp.ok) {
+    if (cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    for (auto& e : hp.ev)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    hp.ok = true;
+  }
+  return &hp;
+}
+
+// Heads per chunk such that one chunk's attention grid fills whole waves of
+// SMs (one CTA per SM), preferring 4..8 heads; the last chunk may be shorter.
+int pick_heads_per_chunk(int64_t n_rows, int n_heads) {
+  const long long qtiles = (n_rows + 2 * h3::attn::BM - 1) / (2 * h3::attn::BM);
+  const int sms = sm_count();
+  int best = n_heads < 4 ? n_heads : 4;
+  double best_waste = 2.0;
+  for (int hc = 2; hc <= 8 && hc <= n_heads; ++hc) {
+    const long long ctas = qtiles * hc;
+    const double waves = static_cast<double>(ctas) / sms;
+    const double waste = std::ceil(waves) / waves - 1.0;   // idle fraction of the last wave
+    if (waste < best_waste - 1e-9) { best_waste = waste; best = hc; }
+  }
+  return best;
+}
+
+}  // namespace
+
+extern "C" {
+
+h3_status h3_packed_mmrope_attention_host(const h3_segment* segs, int32_t nseg, const int32_t* h_perm,
+                                          const void* h_q, const void* h_k, const void* h_v, void* h_o,
+                                          void* d_work, int64_t n_rows, int32_t n_heads,
+                                          int32_t heads_per_chunk, const h3_rope_cfg* cfg, void* stream) {
+  if (n_rows < 0 || n_heads < 1 || !valid_rope_cfg(cfg)) return H3_ERR_INVALID_ARG;
+  if (cfg->head_dim != 128) return H3_ERR_UNSUPPORTED;
+  if (heads_per_chunk < 0 || heads_per_chunk > n_heads) return H3_ERR_INVALID_ARG;
+  if (n_rows == 0) return h3_build_coords(segs, nseg, nullptr, 0, nullptr, stream);
+  if (!h_q || !h_k || !h_v || !h_o) return H3_ERR_INVALID_ARG;
+  if (d_work == nullptr || (reinterpret_cast<uintptr_t>(d_work) & 255u)) return H3_ERR_INVALID_ARG;
+  HostPipe* hp = host_pipe();
+  if (hp == nullptr) return H3_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(hp->enqueue);
+  cudaStream_t s = as_stream(stream);
+
+  // carve the workspace
+  auto up = [](uint64_t b) { return (b + 255u) & ~uint64_t(255u); };
+  const uint64_t row_bytes = static_cast<uint64_t>(n_heads) * 256u;
+  const uint64_t t = up(static_cast<uint64_t>(n_rows) * row_bytes);
+  uint8_t* w = static_cast<uint8_t*>(d_work);
+  uint8_t *dq = w, *dk = w + t, *dv = w + 2 * t, *d_o = w + 3 * t;
+  float* dcoords = reinterpret_cast<float*>(w + 4 * t);
+  int32_t* dperm = reinterpret_cast<int32_t*>(w + 4 * t + up(static_cast<uint64_t>(n_rows) * 12u));
+
+  const int hc = heads_per_chunk > 0 ? heads_per_chunk : pick_heads_per_chunk(n_rows, n_heads);
+  const int nchunks = (n_heads + hc - 1) / hc;
+  if (nchunks > 64) return H3_ERR_UNSUPPORTED;
+  cudaEvent_t* ev_in = hp->ev;
+  cudaEvent_t* ev_out = hp->ev + 64;
+  cudaEvent_t ev_start = hp->ev[192], ev_end = hp->ev[193];
+  auto ck = [](cudaError_t e) { return e == cudaSuccess; };
+
+  // both copy streams start after the work already queued on `stream`
+  if (!ck(cudaEventRecord(ev_start, s)) || !ck(cudaStreamWaitEvent(hp->h2d, ev_start, 0)) ||
+      !ck(cudaStreamWaitEvent(hp->d2h, ev_start, 0)))
+    return H3_ERR_CUDA;
+  // coordinates (after the permutation is on the device)
+  if (h_perm != nullptr) {
+    if (!ck(cudaMemcpyAsync(dperm, h_perm, static_cast<size_t>(n_rows) * 4, cudaMemcpyHostToDevice, s)))
+      return H3_ERR_CUDA;
+  }
+  h3_status st = h3_build_coords(segs, nseg, h_perm ? dperm : nullptr, n_rows, dcoords, stream);
+  if (st != H3_OK) return st;
+
+  for (int c = 0; c < nchunks; ++c) {
+    const int h0 = c * hc, nh = (h0 + hc <= n_heads) ? hc : n_heads - h0;
+    const size_t off = static_cast<size_t>(h0) * 256u, width = static_cast<size_t>(nh) * 256u;
+    for (int x = 0; x < 3; ++x) {
+      const uint8_t* src = static_cast<const uint8_t*>(x == 0 ? h_q : x == 1 ? h_k : h_v) + off;
+      uint8_t* dst = (x == 0 ? dq : x == 1 ? dk : dv) + off;
+      if (!ck(cudaMemcpy2DAsync(dst, row_bytes, src, row_bytes, width, static_cast<size_t>(n_rows),
+                                cudaMemcpyHostToDevice, hp->h2d)))
+        return H3_ERR_CUDA;
+    }
+    if (!ck(cudaEventRecord(ev_in[c], hp->h2d)) || !ck(cudaStreamWaitEvent(s, ev_in[c], 0))) return H3_ERR_CUDA;
+    // rotate this chunk's Q and K in place, then attend over all rows for its heads
+    st = h3_mmrope_qk(dq + off, dk + off, dq + off, dk + off, dcoords, n_rows, nh,
+                      static_cast<int64_t>(n_heads) * 128, cfg, stream);
+    if (st != H3_OK) return st;
+    st = h3_packed_attention(dq + off, dk + off, dv + off, d_o + off, nullptr, nullptr, nullptr, 1, n_rows, nh, 128,
+                             static_cast<int64_t>(n_heads) * 128, 0.f, stream);
+    if (st != H3_OK) return st;
+    if (!ck(cudaEventRecord(ev_out[c], s)) || !ck(cudaStreamWaitEvent(hp->d2h, ev_out[c], 0))) return H3_ERR_CUDA;
+    if (!ck(cudaMemcpy2DAsync(static_cast<uint8_t*>(h_o) + off, row_bytes, d_o + off, row_bytes, width,
+                              static_cast<size_t>(n_rows), cudaMemcpyDeviceToHost, hp->d2h)))
+      return H3_ERR_CUDA;
+  }
+  // `stream` is ordered after the last copy out (and, through it, all others)
+  if (!ck(cudaEventRecord(ev_end, hp->d2h)) || !ck(cudaStreamWaitEvent(s, ev_end, 0))) return H3_ERR_CUDA;
+  return H3_OK;
+}
+
 h3_status h3_check_device_error(void* stream) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return H3_ERR_CUDA;
   unsigned int word = 0, zero = 0;

@@ -27,6 +27,8 @@ def test_every_declared_symbol_is_exported():
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_lib.EXPORTED)
+    assert h3.h3_host_workspace_bytes(100, 2) == 4 * 51200 + 1280 + 512
+    assert h3.h3_host_workspace_bytes(0, 2) == 0
 
 
 def test_struct_layouts_match_header():
