@@ -8,8 +8,10 @@ step of the path runs in the library's CUDA kernels:
 * ``h3_mmrope_qk``        three-axis rotary rotation of bf16 Q and K
 * ``h3_packed_attention`` full softmax attention over the packed rows
 
-Importing the package loads the library and raises if it is missing; there is
-no CPU or eager-PyTorch fallback.
+The library is loaded on first use (``load()``, or any call below) and a
+missing or stale ``libh3.so`` raises there; there is no CPU or eager-PyTorch
+fallback.  Importing the package itself does not load it, so that
+``python -m packed_mm_rope_b200.build`` can (re)build a missing library.
 """
 from __future__ import annotations
 
@@ -19,7 +21,7 @@ from ._lib import (H3Error, H3_OK, H3_ERR_INVALID_ARG, H3_ERR_UNSUPPORTED, H3_ER
                    h3_host_workspace_bytes, h3_mmrope_qk, h3_packed_attention, h3_packed_mmrope_attention_host,
                    h3_set_wait_limit_ns, rope_cfg, status_str)
 
-LIB = _lib.load()
+load = _lib.load
 
 
 def _stream(stream=None) -> int:
