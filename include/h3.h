@@ -54,7 +54,8 @@ typedef enum {
   H3_ERR_UNSUPPORTED = 2,   /* valid but not implemented (head_dim != 128, misalignment, ...) */
   H3_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
   H3_ERR_TIMEOUT = 4,       /* a bounded device-side wait expired (see h3_set_wait_limit_ns) */
-  H3_ERR_DEVICE_INPUT = 5   /* a kernel found a bad input (e.g. perm entry out of range) */
+  H3_ERR_DEVICE_INPUT = 5,  /* a kernel found a bad input (e.g. perm entry out of range) */
+  H3_ERR_TOO_LARGE = 6      /* problem needs more than the fixed scratch of the no-allocation call */
 } h3_status;
 
 /* Segment kinds. */
@@ -244,6 +245,45 @@ h3_status h3_packed_mmrope_attention_host(const h3_segment* segs, int32_t nseg, 
                                           const void* h_q, const void* h_k, const void* h_v, void* h_o,
                                           void* d_work, int64_t n_rows, int32_t n_heads,
                                           int32_t heads_per_chunk, const h3_rope_cfg* cfg, void* stream);
+
+/* Size of the fixed device scratch used by h3_packed_mmrope_attention_host_noalloc. */
+#define H3_NOALLOC_SCRATCH_BYTES (64ull << 20)
+
+/*
+ * h3_packed_mmrope_attention_host_noalloc -- the same computation as
+ * h3_packed_mmrope_attention_host, for callers that cannot allocate device
+ * memory themselves.  The pages describe no such call; it exists for
+ * integration.  Typical callers that cannot allocate: code running inside a
+ * host framework that owns the device's memory pool and does not allow raw
+ * cudaMalloc next to it; latency-bound loops where an allocation (which can
+ * synchronise the device) is not acceptable; plugins that are handed pointers
+ * but no allocator.
+ *
+ * Instead of a caller-provided workspace it uses one fixed scratch array of
+ * H3_NOALLOC_SCRATCH_BYTES (64 MiB) that lives in the library's device code:
+ * every GPU that loads the library holds this memory until the process exits.
+ * The call allocates nothing: no cudaMalloc, no cudaFree, no streams, no
+ * events; all copies and kernels are queued in order on `stream` (no overlap
+ * between copies and compute, unlike the workspace variant).
+ *
+ *   arguments      as h3_packed_mmrope_attention_host, without d_work and
+ *                  heads_per_chunk
+ *   size limit     h3_host_workspace_bytes(n_rows, n_heads) must not exceed
+ *                  H3_NOALLOC_SCRATCH_BYTES, else H3_ERR_TOO_LARGE and nothing
+ *                  is queued (about 65k row-heads: e.g. 4,584 rows x 8 heads)
+ *   first call     the first call on each device looks up the scratch
+ *                  array's device address (cudaGetSymbolAddress) and caches
+ *                  it; make that first call before any stream capture
+ *   sharing        every call on a device uses the same scratch and leaves its
+ *                  contents behind; nothing in it has to start at zero (each
+ *                  call writes every byte it later reads).  Calls whose GPU
+ *                  work overlaps in time (different streams, or different host
+ *                  threads) race on the scratch: serialise them.
+ */
+h3_status h3_packed_mmrope_attention_host_noalloc(const h3_segment* segs, int32_t nseg, const int32_t* h_perm,
+                                                  const void* h_q, const void* h_k, const void* h_v, void* h_o,
+                                                  int64_t n_rows, int32_t n_heads, const h3_rope_cfg* cfg,
+                                                  void* stream);
 
 /*
  * Synchronise `stream`, then read and clear this device's error word.

@@ -12,14 +12,17 @@ import os
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libh3.so")
 
-H3_OK, H3_ERR_INVALID_ARG, H3_ERR_UNSUPPORTED, H3_ERR_CUDA, H3_ERR_TIMEOUT, H3_ERR_DEVICE_INPUT = range(6)
+(H3_OK, H3_ERR_INVALID_ARG, H3_ERR_UNSUPPORTED, H3_ERR_CUDA, H3_ERR_TIMEOUT, H3_ERR_DEVICE_INPUT,
+ H3_ERR_TOO_LARGE) = range(7)
+H3_NOALLOC_SCRATCH_BYTES = 64 << 20
 H3_SEG_TEXT, H3_SEG_VIDEO, H3_SEG_AUDIO = 0, 1, 2
 H3_FLAG_TEXT_T_ONLY, H3_FLAG_AUDIO_CHANNEL_H, H3_FLAG_VIDEO_CANVAS = 1, 2, 4
 H3_MAX_SEGMENTS = 64
 
 EXPORTED = ("h3_status_str", "h3_version", "h3_build_coords", "h3_mmrope_qk",
             "h3_packed_attention", "h3_check_device_error", "h3_set_wait_limit_ns",
-            "h3_host_workspace_bytes", "h3_packed_mmrope_attention_host")
+            "h3_host_workspace_bytes", "h3_packed_mmrope_attention_host",
+            "h3_packed_mmrope_attention_host_noalloc")
 
 
 class h3_segment(ctypes.Structure):
@@ -71,6 +74,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.h3_packed_mmrope_attention_host.restype = I32
     lib.h3_packed_mmrope_attention_host.argtypes = [ctypes.POINTER(h3_segment), I32, P, P, P, P, P, P, I64, I32,
                                                     I32, ctypes.POINTER(h3_rope_cfg), P]
+    lib.h3_packed_mmrope_attention_host_noalloc.restype = I32
+    lib.h3_packed_mmrope_attention_host_noalloc.argtypes = [ctypes.POINTER(h3_segment), I32, P, P, P, P, P, I64,
+                                                            I32, ctypes.POINTER(h3_rope_cfg), P]
     _lib = lib
     return lib
 
@@ -132,6 +138,16 @@ def h3_packed_mmrope_attention_host(segments, h_perm: int, h_q: int, h_k: int, h
                                                   h_v or None, h_o or None, d_work or None, n_rows, n_heads,
                                                   heads_per_chunk, ctypes.byref(cfg), stream or None),
            "h3_packed_mmrope_attention_host")
+
+
+def h3_packed_mmrope_attention_host_noalloc(segments, h_perm: int, h_q: int, h_k: int, h_v: int, h_o: int,
+                                            n_rows: int, n_heads: int, cfg: h3_rope_cfg, stream: int = 0) -> None:
+    """The host-buffer call without a caller workspace (see include/h3.h)."""
+    arr = segment_array(segments)
+    _check(load().h3_packed_mmrope_attention_host_noalloc(arr, len(segments), h_perm or None, h_q or None,
+                                                          h_k or None, h_v or None, h_o or None, n_rows, n_heads,
+                                                          ctypes.byref(cfg), stream or None),
+           "h3_packed_mmrope_attention_host_noalloc")
 
 
 def h3_check_device_error(stream: int = 0) -> int:

@@ -100,6 +100,7 @@ const char* h3_status_str(int32_t status) {
     case H3_ERR_CUDA: return "CUDA error";
     case H3_ERR_TIMEOUT: return "bounded device wait expired";
     case H3_ERR_DEVICE_INPUT: return "kernel found an invalid input";
+    case H3_ERR_TOO_LARGE: return "problem exceeds the fixed scratch of the no-allocation call";
     default: return "unknown status";
   }
 }
@@ -371,6 +372,80 @@ h3_status h3_packed_mmrope_attention_host(const h3_segment* segs, int32_t nseg, 
   }
   // `stream` is ordered after the last copy out (and, through it, all others)
   if (!ck(cudaEventRecord(ev_end, hp->d2h)) || !ck(cudaStreamWaitEvent(s, ev_end, 0))) return H3_ERR_CUDA;
+  return H3_OK;
+}
+
+}  // extern "C"
+
+// ---- allocation-free variant of the host-buffer call ----------------------
+//
+// Its workspace is this file-scope device array instead of caller memory.  In
+// host code the name is only a host-side stand-in for the device symbol: its
+// device address must be looked up with cudaGetSymbolAddress (once per device,
+// with that device current) and that address passed to the kernels.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[H3_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of g_noalloc_scratch on the current device (cached per
+// device after the first lookup), or null if the lookup fails.
+void* noalloc_scratch() {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+h3_status h3_packed_mmrope_attention_host_noalloc(const h3_segment* segs, int32_t nseg, const int32_t* h_perm,
+                                                  const void* h_q, const void* h_k, const void* h_v, void* h_o,
+                                                  int64_t n_rows, int32_t n_heads, const h3_rope_cfg* cfg,
+                                                  void* stream) {
+  if (n_rows < 0 || n_heads < 1 || !valid_rope_cfg(cfg)) return H3_ERR_INVALID_ARG;
+  if (cfg->head_dim != 128) return H3_ERR_UNSUPPORTED;
+  if (n_rows == 0) return h3_build_coords(segs, nseg, nullptr, 0, nullptr, stream);
+  if (!h_q || !h_k || !h_v || !h_o) return H3_ERR_INVALID_ARG;
+  const uint64_t need = h3_host_workspace_bytes(n_rows, n_heads);
+  if (need == 0) return H3_ERR_INVALID_ARG;
+  if (need > H3_NOALLOC_SCRATCH_BYTES) return H3_ERR_TOO_LARGE;
+  uint8_t* w = static_cast<uint8_t*>(noalloc_scratch());
+  if (w == nullptr) return H3_ERR_CUDA;
+
+  // same carving as the workspace variant
+  auto up = [](uint64_t b) { return (b + 255u) & ~uint64_t(255u); };
+  const uint64_t bytes = static_cast<uint64_t>(n_rows) * n_heads * 256u;
+  const uint64_t t = up(bytes);
+  uint8_t *dq = w, *dk = w + t, *dv = w + 2 * t, *d_o = w + 3 * t;
+  float* dcoords = reinterpret_cast<float*>(w + 4 * t);
+  int32_t* dperm = reinterpret_cast<int32_t*>(w + 4 * t + up(static_cast<uint64_t>(n_rows) * 12u));
+  cudaStream_t s = as_stream(stream);
+  const int64_t rs = static_cast<int64_t>(n_heads) * 128;
+
+  // everything in order on `stream`: copies in, coords, rope, attention, copy out
+  if (h_perm != nullptr &&
+      cudaMemcpyAsync(dperm, h_perm, static_cast<size_t>(n_rows) * 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return H3_ERR_CUDA;
+  if (cudaMemcpyAsync(dq, h_q, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dk, h_k, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dv, h_v, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return H3_ERR_CUDA;
+  h3_status st = h3_build_coords(segs, nseg, h_perm ? dperm : nullptr, n_rows, dcoords, stream);
+  if (st != H3_OK) return st;
+  st = h3_mmrope_qk(dq, dk, dq, dk, dcoords, n_rows, n_heads, rs, cfg, stream);
+  if (st != H3_OK) return st;
+  st = h3_packed_attention(dq, dk, dv, d_o, nullptr, nullptr, nullptr, 1, n_rows, n_heads, 128, rs, 0.f, stream);
+  if (st != H3_OK) return st;
+  if (cudaMemcpyAsync(h_o, d_o, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return H3_ERR_CUDA;
   return H3_OK;
 }
 
