@@ -288,11 +288,39 @@ def run_ours(args):
         "gpu_launches": 3 * args.steps,
         "clocks": clk.summary(),
     }
+    if args.adaln:
+        line["adaln"] = time_adaln(h3, wl, dev, stream, pk["hbm_gbs"], args.steps)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, q, k, v, perm, rows=args.cpu_rows)
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def time_adaln(h3, wl, dev, stream, hbm_gbs, steps):
+    """h3_adaln_modulate on the workload's layer input [N, H*128] (not part of the step)."""
+    import torch
+    import workload as W
+    n, c = wl.n_rows, wl.heads * wl.head_dim
+    x = torch.from_numpy(W.normal_bf16(wl.seed, 9, (n, c)).view(np.int16)).view(torch.bfloat16).to(dev)
+    tags = torch.tensor(sum(([s.kind] * s.rows for s in wl.segments), []), dtype=torch.int32, device=dev)
+    ts = torch.zeros(n, dtype=torch.int32, device=dev)
+    table = torch.randn((3, 2, c), dtype=torch.float32, device=dev) * 0.1
+    y = torch.empty_like(x)
+    for _ in range(3):
+        h3.adaln_modulate(x, ts, tags, table, out=y, stream=stream)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        h3.adaln_modulate(x, ts, tags, table, out=y, stream=stream)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b) / steps
+    nbytes = 2 * n * c * 2 + n * 8
+    return {"kernel": "h3_adaln_modulate", "ms": round(ms, 4), "bound": "hbm",
+            "achieved": round(nbytes / (ms * 1e-3) / 1e9, 1), "unit": "GB/s", "peak": hbm_gbs,
+            "frac": round(nbytes / (ms * 1e-3) / 1e9 / hbm_gbs, 4),
+            "algorithmic": "2*N*C*2 + 8*N = %d bytes per launch (x read, y written, two int32 indices)" % nbytes}
 
 
 def profiled_traffic(wl):
@@ -383,6 +411,7 @@ def main():
                     help="resize the worked-example layout to this many latent frames (profiling cases)")
     ap.add_argument("--fused-q-rope", action="store_true",
                     help="rotate only K in h3_mmrope_qk and Q inside h3_packed_attention")
+    ap.add_argument("--adaln", action="store_true", help="also time h3_adaln_modulate on [N, H*128]")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=128, help="query rows of the timed oracle sample")
     ap.add_argument("--ref-rows", type=int, default=16, help="query rows per reference-arm step")

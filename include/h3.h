@@ -207,6 +207,33 @@ h3_status h3_packed_attention(const void* d_q, const void* d_k, const void* d_v,
                               int64_t row_stride, float softmax_scale, void* stream);
 
 /*
+ * h3_adaln_modulate -- per-row AdaLN modulation of the layer input, the step
+ * before the attention projections:  y = LayerNorm(x) * (1 + scale[e]) + shift[e]
+ * with e = timestep_index[row] * 3 + token_tag[row].
+ * Defining passages: [P3] AdaLN passage (computed scale and shift; a table
+ * indexed by (noise level, modality) with adaln_indices = timestep_indices * 3
+ * + token_tags, looked up per row); [P1] section 5 (a small table of unique
+ * timesteps and modalities, gathered for each row).
+ *
+ *   d_x, d_y           device bf16 [n_rows][hidden] with row strides x_row_stride,
+ *                      y_row_stride (elements, multiples of 8; 16-byte aligned);
+ *                      d_y may equal d_x (in place)
+ *   d_timestep_index   device int32[n_rows]; d_token_tag device int32[n_rows]
+ *                      (0 text, 1 video, 2 audio)
+ *   d_table            device fp32 [n_entries][2][hidden]: [e][0] = shift,
+ *                      [e][1] = scale
+ *   eps                LayerNorm epsilon (biased variance; no affine of its own)
+ * Arithmetic: fp32 statistics and modulation, output rounded to bf16.  A row
+ * whose e falls outside [0, n_entries) gets NaN and H3_ERR_DEVICE_INPUT is
+ * reported by h3_check_device_error.
+ * Errors: H3_ERR_INVALID_ARG (sizes, NULL pointers, eps); H3_ERR_UNSUPPORTED
+ * (hidden not a multiple of 8 or above 8192, misaligned pointer or stride).
+ */
+h3_status h3_adaln_modulate(const void* d_x, void* d_y, const int32_t* d_timestep_index,
+                            const int32_t* d_token_tag, const float* d_table, int32_t n_entries, int64_t n_rows,
+                            int32_t hidden, int64_t x_row_stride, int64_t y_row_stride, float eps, void* stream);
+
+/*
  * Device workspace, in bytes, that h3_packed_mmrope_attention_host needs for
  * n_rows x n_heads (Q, K, V, O copies, coordinates and the permutation,
  * each 256-byte aligned).  Returns 0 for invalid sizes.

@@ -17,7 +17,8 @@ from __future__ import annotations
 
 from . import _lib
 from ._lib import (H3Error, H3_OK, H3_ERR_INVALID_ARG, H3_ERR_UNSUPPORTED, H3_ERR_CUDA,  # noqa: F401
-                   H3_ERR_TIMEOUT, H3_ERR_DEVICE_INPUT, h3_build_coords, h3_check_device_error,
+                   H3_ERR_TIMEOUT, H3_ERR_DEVICE_INPUT, H3_ERR_TOO_LARGE, h3_adaln_modulate,
+                   h3_build_coords, h3_check_device_error,
                    h3_host_workspace_bytes, h3_mmrope_qk, h3_packed_attention, h3_packed_mmrope_attention_host,
                    h3_set_wait_limit_ns, rope_cfg, status_str)
 
@@ -167,4 +168,26 @@ def packed_mmrope_attention_host(segments, q, k, v, out=None, perm=None, workspa
                                     k.data_ptr(), v.data_ptr(), out.data_ptr(), workspace.data_ptr(), n, h,
                                     rope_cfg(theta, 128, sections, pair_layout), heads_per_chunk,
                                     _stream(stream))
+    return out
+
+
+def adaln_modulate(x, timestep_index, token_tag, table, out=None, eps: float = 1e-6, stream=None):
+    """y = LayerNorm(x) * (1 + scale[e]) + shift[e], e = timestep_index * 3 + token_tag.
+
+    x: CUDA bf16 [N, C] (row stride a multiple of 8); timestep_index, token_tag:
+    CUDA int32 [N]; table: CUDA fp32 [E, 2, C] (shift, scale).  Pass out=x for in place.
+    """
+    import torch
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1 or not x.is_cuda:
+        raise ValueError("x must be a CUDA bf16 [N, C] tensor with unit inner stride")
+    n, c = x.shape
+    out = torch.empty_like(x) if out is None else out
+    for t in (timestep_index, token_tag):
+        if t.dtype != torch.int32 or t.numel() != n or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError("indices must be contiguous CUDA int32 [N]")
+    if table.dtype != torch.float32 or table.dim() != 3 or tuple(table.shape[1:]) != (2, c) \
+            or not table.is_contiguous():
+        raise ValueError("table must be contiguous fp32 [E, 2, C]")
+    h3_adaln_modulate(x.data_ptr(), out.data_ptr(), timestep_index.data_ptr(), token_tag.data_ptr(),
+                      table.data_ptr(), table.shape[0], n, c, x.stride(0), out.stride(0), eps, _stream(stream))
     return out

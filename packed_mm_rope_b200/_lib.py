@@ -22,7 +22,7 @@ H3_MAX_SEGMENTS = 64
 EXPORTED = ("h3_status_str", "h3_version", "h3_build_coords", "h3_mmrope_qk",
             "h3_packed_attention", "h3_check_device_error", "h3_set_wait_limit_ns",
             "h3_host_workspace_bytes", "h3_packed_mmrope_attention_host",
-            "h3_packed_mmrope_attention_host_noalloc")
+            "h3_packed_mmrope_attention_host_noalloc", "h3_adaln_modulate")
 
 
 class h3_segment(ctypes.Structure):
@@ -77,6 +77,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.h3_packed_mmrope_attention_host_noalloc.restype = I32
     lib.h3_packed_mmrope_attention_host_noalloc.argtypes = [ctypes.POINTER(h3_segment), I32, P, P, P, P, P, I64,
                                                             I32, ctypes.POINTER(h3_rope_cfg), P]
+    lib.h3_adaln_modulate.restype = I32
+    lib.h3_adaln_modulate.argtypes = [P, P, P, P, P, I32, I64, I32, I64, I64, F32, P]
     _lib = lib
     return lib
 
@@ -148,6 +150,13 @@ def h3_packed_mmrope_attention_host_noalloc(segments, h_perm: int, h_q: int, h_k
                                                           h_k or None, h_v or None, h_o or None, n_rows, n_heads,
                                                           ctypes.byref(cfg), stream or None),
            "h3_packed_mmrope_attention_host_noalloc")
+
+
+def h3_adaln_modulate(d_x: int, d_y: int, d_ts: int, d_tags: int, d_table: int, n_entries: int, n_rows: int,
+                      hidden: int, x_row_stride: int, y_row_stride: int, eps: float = 1e-6, stream: int = 0) -> None:
+    _check(load().h3_adaln_modulate(d_x or None, d_y or None, d_ts or None, d_tags or None, d_table or None,
+                                    n_entries, n_rows, hidden, x_row_stride, y_row_stride, eps, stream or None),
+           "h3_adaln_modulate")
 
 
 def h3_check_device_error(stream: int = 0) -> int:

@@ -3,6 +3,7 @@
 // Host-side argument validation, TMA tensor-map encoding and kernel launches.
 // The library allocates no device memory; the per-device error word is a
 // static __device__ variable of this module.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -12,6 +13,7 @@
 #include "coords.cuh"
 #include "rope.cuh"
 #include "attention.cuh"
+#include "adaln.cuh"
 
 namespace {
 
@@ -242,6 +244,36 @@ h3_status h3_packed_attention(const void* d_q, const void* d_k, const void* d_v,
                   static_cast<unsigned>(n_heads), static_cast<unsigned>(batch));
   h3::attn::attention_kernel<<<grid, h3::attn::THREADS, h3::attn::SMEM_BYTES, as_stream(stream)>>>(tq, tk, tv,
                                                                                                   p);
+  return cudaGetLastError() == cudaSuccess ? H3_OK : H3_ERR_CUDA;
+}
+
+h3_status h3_adaln_modulate(const void* d_x, void* d_y, const int32_t* d_timestep_index,
+                            const int32_t* d_token_tag, const float* d_table, int32_t n_entries, int64_t n_rows,
+                            int32_t hidden, int64_t x_row_stride, int64_t y_row_stride, float eps, void* stream) {
+  if (n_rows < 0 || hidden < 8 || n_entries < 1 || !(eps >= 0.f) || !std::isfinite(eps)) return H3_ERR_INVALID_ARG;
+  if (hidden % 8 != 0 || hidden > h3::ADALN_MAX_HIDDEN) return H3_ERR_UNSUPPORTED;
+  if (x_row_stride < hidden || y_row_stride < hidden) return H3_ERR_INVALID_ARG;
+  if (n_rows == 0) return H3_OK;
+  if (!d_x || !d_y || !d_timestep_index || !d_token_tag || !d_table) return H3_ERR_INVALID_ARG;
+  if (x_row_stride % 8 || y_row_stride % 8 || !aligned16(d_x) || !aligned16(d_y) || !aligned16(d_table))
+    return H3_ERR_UNSUPPORTED;
+  const size_t smem = h3::adaln_smem_bytes(hidden);
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    size_t most = 0;
+    for (int hdn = 8; hdn <= h3::ADALN_MAX_HIDDEN; hdn += 8) most = std::max(most, h3::adaln_smem_bytes(hdn));
+    attr_err = cudaFuncSetAttribute(h3::adaln_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(most));
+  });
+  if (attr_err != cudaSuccess) return H3_ERR_CUDA;
+  // one CTA per SM (the rings fill shared memory); contiguous row blocks
+  const long long grid = std::min<long long>(sm_count(), (n_rows + h3::ADALN_WARPS - 1) / h3::ADALN_WARPS);
+  const long long per_cta = (n_rows + grid - 1) / grid;
+  h3::adaln_kernel<<<static_cast<int>(grid), h3::ADALN_THREADS, smem, as_stream(stream)>>>(
+      static_cast<const uint4*>(d_x), static_cast<uint4*>(d_y), d_timestep_index, d_token_tag,
+      reinterpret_cast<const float4*>(d_table), n_entries, n_rows, hidden / 8, x_row_stride / 8, y_row_stride / 8,
+      eps, g_wait_limit_ns, per_cta);
   return cudaGetLastError() == cudaSuccess ? H3_OK : H3_ERR_CUDA;
 }
 
