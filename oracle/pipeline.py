@@ -23,26 +23,26 @@ def _as_f64(x: np.ndarray) -> np.ndarray:
     return x.astype(np.float64)
 
 
-def packed_angles(segments, perm, theta, sections):
+def packed_angles(segments, perm, theta, sections, freq_rule=0):
     v64, _ = _coords.packed_values(segments, perm)
-    return _rope.angles(v64, theta, sections)
+    return _rope.angles(v64, theta, sections, freq_rule)
 
 
-def rotated_qk(segments, perm, q, k, theta=10000.0, sections=(32, 48, 48), pair_layout=0):
+def rotated_qk(segments, perm, q, k, theta=10000.0, sections=(32, 48, 48), pair_layout=0, freq_rule=0):
     """fp64 rotated (Q, K), each [N, H, D]."""
-    ang = packed_angles(segments, perm, theta, sections)
+    ang = packed_angles(segments, perm, theta, sections, freq_rule)
     return (_rope.rotate(_as_f64(q), ang, pair_layout),
             _rope.rotate(_as_f64(k), ang, pair_layout))
 
 
 def packed_mmrope_attention(segments, perm, q, k, v, theta=10000.0, sections=(32, 48, 48),
-                            rows=None, heads=None, pair_layout=0, scale=None):
+                            rows=None, heads=None, pair_layout=0, scale=None, freq_rule=0):
     """O [len(rows), len(heads), D] and LSE [len(heads), len(rows)] in fp64."""
     q = np.asarray(q)
     N, H, _ = q.shape
     rows = np.arange(N) if rows is None else np.asarray(rows, np.int64)
     heads = range(H) if heads is None else list(heads)
-    ang = packed_angles(segments, perm, theta, sections)
+    ang = packed_angles(segments, perm, theta, sections, freq_rule)
     o = np.empty((rows.size, len(heads), v.shape[2]), np.float64)
     lse = np.empty((len(heads), rows.size), np.float64)
     for i, h in enumerate(heads):

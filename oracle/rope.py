@@ -7,7 +7,11 @@ Definition followed:
   values and the inverse frequencies are computed from them, not stored.
   Reading used here: the head dimension is split into per-axis sections
   (t:32, h:48, w:48 dims) and axis a with D_a dims has the D_a/2 inverse
-  frequencies theta^(-2j/D_a), j = 0 .. D_a/2 - 1.
+  frequencies theta^(-2j/D_a), j = 0 .. D_a/2 - 1 (freq_rule=0).
+  The alternative reading (freq_rule=1): ``rope_freq_dim`` is the whole head
+  dimension D, so pair p (counted over the head, t pairs first) has the one
+  ladder's frequency theta^(-2p/D) and the sections only say which axis
+  coordinate drives it.
 * Rotary pair layout: adjacent dims (2p, 2p+1) form pair p; pairs 0..15 are
   t, 16..39 are h, 40..63 are w (pair_layout=0).  The alternative half-split
   layout pairs dim p with dim p + D/2 (pair_layout=1).
@@ -19,29 +23,39 @@ from __future__ import annotations
 import numpy as np
 
 
-def inv_freq(theta: float, sections=(32, 48, 48)):
-    """Per-axis inverse frequencies, a list of three fp64 arrays."""
-    out = []
+def inv_freq(theta: float, sections=(32, 48, 48), freq_rule: int = 0):
+    """Inverse frequencies of each axis's pairs, a list of three fp64 arrays.
+
+    freq_rule 0: axis a restarts the ladder, theta^(-2j/D_a) for its D_a/2 pairs.
+    freq_rule 1: one ladder theta^(-2p/D) over all D/2 pairs of the head, cut
+    into the axes' consecutive slices.
+    """
     for d_a in sections:
         if d_a % 2:
             raise ValueError("each axis needs an even number of dims")
-        j = np.arange(d_a // 2, dtype=np.float64)
-        out.append(np.power(np.float64(theta), -2.0 * j / d_a))
-    return out
+    if freq_rule == 0:
+        return [np.power(np.float64(theta), -2.0 * np.arange(d_a // 2, dtype=np.float64) / d_a)
+                for d_a in sections]
+    if freq_rule == 1:
+        D = sum(sections)
+        ladder = np.power(np.float64(theta), -2.0 * np.arange(D // 2, dtype=np.float64) / D)
+        cut = np.cumsum([0] + [d_a // 2 for d_a in sections])
+        return [ladder[cut[a]:cut[a + 1]] for a in range(len(sections))]
+    raise ValueError("freq_rule must be 0 or 1")
 
 
-def pair_table(theta: float, sections=(32, 48, 48)):
+def pair_table(theta: float, sections=(32, 48, 48), freq_rule: int = 0):
     """(axis[p], inv_freq[p]) for every rotary pair p = 0 .. D/2 - 1."""
     axes, freqs = [], []
-    for a, f in enumerate(inv_freq(theta, sections)):
+    for a, f in enumerate(inv_freq(theta, sections, freq_rule)):
         axes.append(np.full(f.size, a, np.int64))
         freqs.append(f)
     return np.concatenate(axes), np.concatenate(freqs)
 
 
-def angles(coords: np.ndarray, theta: float, sections=(32, 48, 48)) -> np.ndarray:
+def angles(coords: np.ndarray, theta: float, sections=(32, 48, 48), freq_rule: int = 0) -> np.ndarray:
     """[rows, D/2] rotation angle of every pair: coords[r, axis[p]] * inv_freq[p]."""
-    axis, freq = pair_table(theta, sections)
+    axis, freq = pair_table(theta, sections, freq_rule)
     return np.asarray(coords, np.float64)[:, axis] * freq[None, :]
 
 

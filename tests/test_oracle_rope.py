@@ -141,3 +141,54 @@ def test_pipeline_rotated_qk_uses_packed_coords():
     # the permuted row r carries logical element perm[r]'s coordinates
     numl, denl = coords.logical_coords(wl.segments)
     assert (num == numl[perm]).all()
+
+
+# ---- the single-ladder frequency reading (freq_rule=1) ----------------------
+
+def test_single_ladder_pair_table():
+    axis0, _ = rope.pair_table(THETA, SECTIONS)
+    axis, freq = rope.pair_table(THETA, SECTIONS, freq_rule=1)
+    assert (axis == axis0).all(), "the sections still assign the axes"
+    # one geometric ladder over the whole head, no restart at the section edges
+    assert freq[0] == 1.0
+    np.testing.assert_allclose(freq[1:] / freq[:-1], THETA ** (-2.0 / 128), rtol=1e-14)
+    np.testing.assert_allclose(freq[16], THETA ** (-32.0 / 128), rtol=1e-14)   # first h pair
+    np.testing.assert_allclose(freq[40], THETA ** (-80.0 / 128), rtol=1e-14)   # first w pair
+
+
+def test_single_ladder_text_is_full_head_1d_rope():
+    # text rows sit at (i, i, i): with one ladder every pair sees the same
+    # coordinate, which is textbook 1-D RoPE over all 128 dims
+    n = 24
+    x = _rng(11).standard_normal((n, 2, 128))
+    num, den = coords.logical_coords([W.text(n)])
+    ang = rope.angles(coords.to_f64(num, den), THETA, SECTIONS, freq_rule=1)
+    y0 = rope.rotate(x, ang, pair_layout=0)
+    y1 = rope.rotate(x, ang, pair_layout=1)
+    for i in range(n):
+        for h in range(2):
+            np.testing.assert_allclose(y0[i, h], _complex_rope_1d(x[i, h], i, 128, 128), atol=1e-12)
+            for p in range(64):
+                z = complex(x[i, h, p], x[i, h, p + 64]) * cmath.exp(1j * i * THETA ** (-2.0 * p / 128))
+                assert abs(y1[i, h, p] - z.real) < 1e-12 and abs(y1[i, h, p + 64] - z.imag) < 1e-12
+
+
+def test_single_ladder_relative_form():
+    rng = _rng(12)
+    for _ in range(10):
+        q, k = rng.standard_normal(128), rng.standard_normal(128)
+        pq, pk = rng.uniform(-50, 50, 3), rng.uniform(-50, 50, 3)
+        qr = rope.rotate(q[None], rope.angles(pq[None], THETA, SECTIONS, 1))[0]
+        kr = rope.rotate(k[None], rope.angles(pk[None], THETA, SECTIONS, 1))[0]
+        d = pk - pq
+        R = np.zeros((128, 128))
+        for p in range(64):
+            a = d[0 if p < 16 else 1 if p < 40 else 2] * THETA ** (-p / 64.0)
+            R[2 * p:2 * p + 2, 2 * p:2 * p + 2] = [[math.cos(a), -math.sin(a)], [math.sin(a), math.cos(a)]]
+        assert abs(qr @ kr - q @ R @ k) < 1e-10
+
+
+def test_unknown_freq_rule_is_an_error():
+    import pytest
+    with pytest.raises(ValueError):
+        rope.inv_freq(THETA, SECTIONS, freq_rule=2)
