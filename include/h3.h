@@ -109,10 +109,16 @@ typedef struct {
 /*
  * Rotary configuration ([P3] rope-config passage; [P5] H3-Omni-Transformer).
  * The head dimension is split into per-axis sections sec_t + sec_h + sec_w
- * == head_dim (each even); axis a with D_a dims rotates D_a/2 pairs with
- * inverse frequencies theta^(-2j / D_a), j = 0 .. D_a/2 - 1, computed in fp64.
- * pair_layout 0: pair p = dims (2p, 2p+1); pairs [0, sec_t/2) are t, then h,
- * then w.  pair_layout 1: pair p = dims (p, p + head_dim/2), same axis order.
+ * == head_dim (each even); pairs [0, sec_t/2) are driven by t, the next
+ * sec_h/2 by h, the last sec_w/2 by w.
+ * freq_rule 0 (default): axis a with D_a dims restarts the frequency ladder,
+ *   its j-th pair has inverse frequency theta^(-2j / D_a).
+ * freq_rule 1: one ladder over the whole head, pair p (counted over the head)
+ *   has theta^(-2p / head_dim).  The pages name a rope frequency dimension
+ *   without a formula; these are its two plain readings.
+ * Frequencies are computed in fp64 on the host.
+ * pair_layout 0: pair p = dims (2p, 2p+1).  pair_layout 1: pair p = dims
+ * (p, p + head_dim/2).
  * A pair (x0, x1) at angle a becomes (x0 cos a - x1 sin a, x0 sin a + x1 cos a).
  */
 typedef struct {
@@ -122,6 +128,7 @@ typedef struct {
   int32_t sec_h;       /* 48 */
   int32_t sec_w;       /* 48 */
   int32_t pair_layout; /* 0 (adjacent, default) or 1 (half-split) */
+  int32_t freq_rule;   /* 0 (per-axis ladders, default) or 1 (one ladder) */
 } h3_rope_cfg;
 
 /* Short English text for a status code (static storage; never NULL). */
@@ -129,6 +136,30 @@ const char* h3_status_str(int32_t status);
 
 /* Library ABI version (major * 100 + minor). */
 int32_t h3_version(void);
+
+/*
+ * h3_init -- optional up-front set-up of one device.  The pages define no
+ * counterpart; it is plumbing.  Checks that `device` exists and has compute
+ * capability 10.0 (the kernels are built for sm_100a only) and that the
+ * kernels load on it, then does once what every other call otherwise does
+ * lazily on first use: the shared-memory opt-ins of the kernels, the lookup of
+ * the driver's tensor-map encoder, the host-buffer pipeline's two streams and
+ * events, the address of the no-allocation scratch; and clears the device
+ * error word.  Allocates no device memory.  The calling thread's current
+ * device is left as it was.  Calling it again is harmless.
+ * Errors: H3_ERR_INVALID_ARG (no such device), H3_ERR_UNSUPPORTED (another
+ * architecture, or the kernels do not load), H3_ERR_CUDA.
+ */
+h3_status h3_init(int32_t device);
+
+/*
+ * h3_shutdown -- releases what the library created: on every device, waits
+ * for and destroys the host-buffer pipeline's streams and events.  Must not
+ * run concurrently with another call of the library.  The library stays
+ * usable: a later call re-creates what it needs.  The calling thread's
+ * current device is left as it was.
+ */
+void h3_shutdown(void);
 
 /*
  * h3_build_coords -- packed segment table -> per-row (t, h, w) fp32.

@@ -18,7 +18,7 @@ from __future__ import annotations
 from . import _lib
 from ._lib import (H3Error, H3_OK, H3_ERR_INVALID_ARG, H3_ERR_UNSUPPORTED, H3_ERR_CUDA,  # noqa: F401
                    H3_ERR_TIMEOUT, H3_ERR_DEVICE_INPUT, H3_ERR_TOO_LARGE, h3_adaln_modulate,
-                   h3_build_coords, h3_check_device_error,
+                   h3_build_coords, h3_check_device_error, h3_init, h3_shutdown,
                    h3_host_workspace_bytes, h3_mmrope_qk, h3_packed_attention, h3_packed_mmrope_attention_host,
                    h3_set_wait_limit_ns, rope_cfg, status_str)
 
@@ -61,7 +61,7 @@ def build_coords(segments, n_rows: int, perm=None, out=None, stream=None):
 
 
 def mmrope_qk(q, k, coords, q_out=None, k_out=None, theta=10000.0, sections=(32, 48, 48), pair_layout=0,
-              stream=None):
+              stream=None, freq_rule=0):
     """Rotate Q and K; returns (q_out, k_out).  Pass q_out=q, k_out=k for in place.
 
     q=None rotates K only (returns (None, k_out)).
@@ -81,12 +81,12 @@ def mmrope_qk(q, k, coords, q_out=None, k_out=None, theta=10000.0, sections=(32,
         raise ValueError("coords must be contiguous fp32 [rows, 3]")
     h3_mmrope_qk(q.data_ptr() if q is not None else 0, k.data_ptr(),
                  q_out.data_ptr() if q is not None else 0, k_out.data_ptr(), coords.data_ptr(), b * n, h,
-                 rs, rope_cfg(theta, 128, sections, pair_layout), _stream(stream))
+                 rs, rope_cfg(theta, 128, sections, pair_layout, freq_rule), _stream(stream))
     return (q_out if q is not None else None), k_out
 
 
 def packed_attention(q, k, v, out=None, lse=None, softmax_scale: float = 0.0, stream=None, coords=None,
-                     theta=10000.0, sections=(32, 48, 48), pair_layout=0):
+                     theta=10000.0, sections=(32, 48, 48), pair_layout=0, freq_rule=0):
     """O = softmax(Q K^T * scale) V over all packed rows, per head.
 
     With ``coords`` (fp32 [rows, 3]) Q is passed UNROTATED and rotated inside
@@ -109,7 +109,7 @@ def packed_attention(q, k, v, out=None, lse=None, softmax_scale: float = 0.0, st
     if coords is not None:
         if coords.dtype != torch.float32 or coords.numel() != 3 * b * n or not coords.is_contiguous():
             raise ValueError("coords must be contiguous fp32 [rows, 3]")
-        cp, cfg = coords.data_ptr(), rope_cfg(theta, 128, sections, pair_layout)
+        cp, cfg = coords.data_ptr(), rope_cfg(theta, 128, sections, pair_layout, freq_rule)
     h3_packed_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lp, b, n, h, rs,
                         softmax_scale, d_coords=cp, cfg=cfg, stream=_stream(stream))
     return out
@@ -117,7 +117,7 @@ def packed_attention(q, k, v, out=None, lse=None, softmax_scale: float = 0.0, st
 
 def packed_mmrope_attention(segments, q, k, v, perm=None, theta=10000.0, sections=(32, 48, 48),
                             pair_layout=0, out=None, lse=None, softmax_scale: float = 0.0, stream=None,
-                            fused_q_rope: bool = False):
+                            fused_q_rope: bool = False, freq_rule=0):
     """The whole path on one packed sequence: coords -> rotate Q, K -> attention.
 
     q, k, v: [N, H, 128] bf16 on the GPU (unrotated).  Returns O [N, H, 128].
@@ -127,10 +127,12 @@ def packed_mmrope_attention(segments, q, k, v, perm=None, theta=10000.0, section
     coords = build_coords(segments, n, perm, stream=stream)
     if fused_q_rope:
         _, kr = mmrope_qk(None, k, coords, theta=theta, sections=sections, pair_layout=pair_layout,
-                          stream=stream)
+                          stream=stream, freq_rule=freq_rule)
         return packed_attention(q, kr, v, out=out, lse=lse, softmax_scale=softmax_scale, stream=stream,
-                                coords=coords, theta=theta, sections=sections, pair_layout=pair_layout)
-    qr, kr = mmrope_qk(q, k, coords, theta=theta, sections=sections, pair_layout=pair_layout, stream=stream)
+                                coords=coords, theta=theta, sections=sections, pair_layout=pair_layout,
+                                freq_rule=freq_rule)
+    qr, kr = mmrope_qk(q, k, coords, theta=theta, sections=sections, pair_layout=pair_layout, stream=stream,
+                       freq_rule=freq_rule)
     return packed_attention(qr, kr, v, out=out, lse=lse, softmax_scale=softmax_scale, stream=stream)
 
 
@@ -144,7 +146,8 @@ def host_workspace(n_rows: int, n_heads: int, device=None):
 
 
 def packed_mmrope_attention_host(segments, q, k, v, out=None, perm=None, workspace=None, theta=10000.0,
-                                 sections=(32, 48, 48), pair_layout=0, heads_per_chunk: int = 0, stream=None):
+                                 sections=(32, 48, 48), pair_layout=0, heads_per_chunk: int = 0, stream=None,
+                                 freq_rule=0):
     """The whole path from and to HOST memory, copies overlapped with compute.
 
     q, k, v: CPU bf16 [N, H, 128] contiguous tensors (pin them for overlap);
@@ -166,7 +169,7 @@ def packed_mmrope_attention_host(segments, q, k, v, out=None, perm=None, workspa
         workspace = host_workspace(n, h)
     h3_packed_mmrope_attention_host(segments, perm.data_ptr() if perm is not None else 0, q.data_ptr(),
                                     k.data_ptr(), v.data_ptr(), out.data_ptr(), workspace.data_ptr(), n, h,
-                                    rope_cfg(theta, 128, sections, pair_layout), heads_per_chunk,
+                                    rope_cfg(theta, 128, sections, pair_layout, freq_rule), heads_per_chunk,
                                     _stream(stream))
     return out
 

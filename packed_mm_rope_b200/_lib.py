@@ -22,7 +22,7 @@ H3_MAX_SEGMENTS = 64
 EXPORTED = ("h3_status_str", "h3_version", "h3_build_coords", "h3_mmrope_qk",
             "h3_packed_attention", "h3_check_device_error", "h3_set_wait_limit_ns",
             "h3_host_workspace_bytes", "h3_packed_mmrope_attention_host",
-            "h3_packed_mmrope_attention_host_noalloc", "h3_adaln_modulate")
+            "h3_packed_mmrope_attention_host_noalloc", "h3_adaln_modulate", "h3_init", "h3_shutdown")
 
 
 class h3_segment(ctypes.Structure):
@@ -32,7 +32,8 @@ class h3_segment(ctypes.Structure):
 
 class h3_rope_cfg(ctypes.Structure):
     _fields_ = [("theta", ctypes.c_double), ("head_dim", ctypes.c_int32), ("sec_t", ctypes.c_int32),
-                ("sec_h", ctypes.c_int32), ("sec_w", ctypes.c_int32), ("pair_layout", ctypes.c_int32)]
+                ("sec_h", ctypes.c_int32), ("sec_w", ctypes.c_int32), ("pair_layout", ctypes.c_int32),
+                ("freq_rule", ctypes.c_int32)]
 
 
 class H3Error(RuntimeError):
@@ -77,6 +78,10 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.h3_packed_mmrope_attention_host_noalloc.restype = I32
     lib.h3_packed_mmrope_attention_host_noalloc.argtypes = [ctypes.POINTER(h3_segment), I32, P, P, P, P, P, I64,
                                                             I32, ctypes.POINTER(h3_rope_cfg), P]
+    lib.h3_init.restype = I32
+    lib.h3_init.argtypes = [I32]
+    lib.h3_shutdown.restype = None
+    lib.h3_shutdown.argtypes = []
     lib.h3_adaln_modulate.restype = I32
     lib.h3_adaln_modulate.argtypes = [P, P, P, P, P, I32, I64, I32, I64, I64, F32, P]
     _lib = lib
@@ -102,9 +107,9 @@ def segment_array(segments):
     return arr
 
 
-def rope_cfg(theta=10000.0, head_dim=128, sections=(32, 48, 48), pair_layout=0) -> h3_rope_cfg:
+def rope_cfg(theta=10000.0, head_dim=128, sections=(32, 48, 48), pair_layout=0, freq_rule=0) -> h3_rope_cfg:
     return h3_rope_cfg(float(theta), int(head_dim), int(sections[0]), int(sections[1]), int(sections[2]),
-                       int(pair_layout))
+                       int(pair_layout), int(freq_rule))
 
 
 def h3_build_coords(segments, d_perm: int, n_rows: int, d_coords: int, stream: int = 0) -> None:
@@ -162,6 +167,16 @@ def h3_adaln_modulate(d_x: int, d_y: int, d_ts: int, d_tags: int, d_table: int, 
 def h3_check_device_error(stream: int = 0) -> int:
     """Synchronise the stream and return (and clear) the device error status."""
     return int(load().h3_check_device_error(stream or None))
+
+
+def h3_init(device: int = 0) -> None:
+    """Up-front set-up of one device (optional; every call also does it lazily)."""
+    _check(load().h3_init(int(device)), "h3_init")
+
+
+def h3_shutdown() -> None:
+    """Release the library's streams and events on every device."""
+    load().h3_shutdown()
 
 
 def h3_set_wait_limit_ns(ns: int) -> None:

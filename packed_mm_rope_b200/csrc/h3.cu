@@ -25,11 +25,40 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
+// One-time set-up of the current device, kept for the life of the process:
+// the shared-memory opt-ins of the kernels that need more than 48 KB
+// (function attributes are per device) and the SM count.
+struct DeviceState {
+  bool ready = false;
+  int sms = 148;
+};
+
+const DeviceState* device_state() {
+  static std::mutex mu;
+  static DeviceState states[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  DeviceState& st = states[dev];
+  if (!st.ready) {
+    size_t adaln_most = 0;
+    for (int hdn = 8; hdn <= h3::ADALN_MAX_HIDDEN; hdn += 8)
+      adaln_most = std::max(adaln_most, h3::adaln_smem_bytes(hdn));
+    if (cudaFuncSetAttribute(h3::attn::attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(h3::attn::SMEM_BYTES)) != cudaSuccess ||
+        cudaFuncSetAttribute(h3::adaln_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(adaln_most)) != cudaSuccess)
+      return nullptr;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) st.sms = n;
+    st.ready = true;
+  }
+  return &st;
+}
+
 int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
-  return n > 0 ? n : 148;
+  const DeviceState* st = device_state();
+  return st ? st->sms : 148;
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -75,6 +104,7 @@ bool valid_rope_cfg(const h3_rope_cfg* cfg) {
   if ((cfg->sec_t | cfg->sec_h | cfg->sec_w) & 1) return false;
   if (cfg->sec_t + cfg->sec_h + cfg->sec_w != cfg->head_dim) return false;
   if (cfg->pair_layout != 0 && cfg->pair_layout != 1) return false;
+  if (cfg->freq_rule != 0 && cfg->freq_rule != 1) return false;
   return true;
 }
 
@@ -84,7 +114,9 @@ h3::RopeTable make_rope_table(const h3_rope_cfg* cfg) {
   int p = 0;
   for (int a = 0; a < 3; ++a)
     for (int j = 0; j < sec[a] / 2; ++j, ++p) {
-      t.inv_freq[p] = std::pow(cfg->theta, -2.0 * j / sec[a]);
+      // per-axis ladder (rule 0) or one ladder over the head's pairs (rule 1)
+      t.inv_freq[p] = cfg->freq_rule == 0 ? std::pow(cfg->theta, -2.0 * j / sec[a])
+                                          : std::pow(cfg->theta, -2.0 * p / cfg->head_dim);
       t.axis[p] = a;
     }
   return t;
@@ -107,7 +139,7 @@ const char* h3_status_str(int32_t status) {
   }
 }
 
-int32_t h3_version(void) { return 100; }
+int32_t h3_version(void) { return 101; }
 
 h3_status h3_set_wait_limit_ns(uint64_t ns) {
   g_wait_limit_ns = ns == 0 ? kDefaultWaitLimitNs : ns;
@@ -216,13 +248,7 @@ h3_status h3_packed_attention(const void* d_q, const void* d_k, const void* d_v,
       !make_qkv_map(&tk, d_k, batch, n_rows, n_heads, row_stride) ||
       !make_qkv_map(&tv, d_v, batch, n_rows, n_heads, row_stride))
     return H3_ERR_CUDA;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(h3::attn::attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(h3::attn::SMEM_BYTES));
-  });
-  if (attr_err != cudaSuccess) return H3_ERR_CUDA;
+  if (device_state() == nullptr) return H3_ERR_CUDA;
 
   h3::attn::Params p;
   p.n_rows = static_cast<int>(n_rows);
@@ -258,15 +284,7 @@ h3_status h3_adaln_modulate(const void* d_x, void* d_y, const int32_t* d_timeste
   if (x_row_stride % 8 || y_row_stride % 8 || !aligned16(d_x) || !aligned16(d_y) || !aligned16(d_table))
     return H3_ERR_UNSUPPORTED;
   const size_t smem = h3::adaln_smem_bytes(hidden);
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    size_t most = 0;
-    for (int hdn = 8; hdn <= h3::ADALN_MAX_HIDDEN; hdn += 8) most = std::max(most, h3::adaln_smem_bytes(hdn));
-    attr_err = cudaFuncSetAttribute(h3::adaln_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(most));
-  });
-  if (attr_err != cudaSuccess) return H3_ERR_CUDA;
+  if (device_state() == nullptr) return H3_ERR_CUDA;
   // one CTA per SM (the rings fill shared memory); contiguous row blocks
   const long long grid = std::min<long long>(sm_count(), (n_rows + h3::ADALN_WARPS - 1) / h3::ADALN_WARPS);
   const long long per_cta = (n_rows + grid - 1) / grid;
@@ -298,9 +316,12 @@ struct HostPipe {
   bool ok = false;
 };
 
+std::mutex g_pipes_mu;
+HostPipe g_pipes[64];
+
 HostPipe* host_pipe() {
-  static std::mutex mu;
-  static HostPipe pipes[64];
+  std::mutex& mu = g_pipes_mu;
+  HostPipe* pipes = g_pipes;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
@@ -313,6 +334,28 @@ HostPipe* host_pipe() {
     hp.ok = true;
   }
   return &hp;
+}
+
+// Waits for and destroys every device's pipeline streams and events; the next
+// host-buffer call re-creates them.  Changes the current device.
+void release_host_pipes() {
+  std::lock_guard<std::mutex> lock(g_pipes_mu);
+  for (int dev = 0; dev < 64; ++dev) {
+    HostPipe& hp = g_pipes[dev];
+    if (!hp.ok) continue;
+    std::lock_guard<std::mutex> q(hp.enqueue);
+    if (cudaSetDevice(dev) != cudaSuccess) continue;
+    cudaStreamSynchronize(hp.h2d);
+    cudaStreamSynchronize(hp.d2h);
+    for (auto& e : hp.ev) {
+      cudaEventDestroy(e);
+      e = nullptr;
+    }
+    cudaStreamDestroy(hp.h2d);
+    cudaStreamDestroy(hp.d2h);
+    hp.h2d = hp.d2h = nullptr;
+    hp.ok = false;
+  }
 }
 
 // Heads per chunk such that one chunk's attention grid fills whole waves of
@@ -490,6 +533,49 @@ h3_status h3_check_device_error(void* stream) {
   if (word & h3::DEVERR_TIMEOUT) return H3_ERR_TIMEOUT;
   if (word & h3::DEVERR_INPUT) return H3_ERR_DEVICE_INPUT;
   return H3_OK;
+}
+
+}  // extern "C"
+
+// ---- lifecycle ------------------------------------------------------------
+
+namespace {
+
+// Restores the calling thread's current device on scope exit.
+struct DeviceGuard {
+  int saved = -1;
+  DeviceGuard() { if (cudaGetDevice(&saved) != cudaSuccess) saved = -1; }
+  ~DeviceGuard() { if (saved >= 0) cudaSetDevice(saved); }
+};
+
+}  // namespace
+
+extern "C" {
+
+h3_status h3_init(int32_t device) {
+  int count = 0;
+  if (cudaGetDeviceCount(&count) != cudaSuccess) return H3_ERR_CUDA;
+  if (device < 0 || device >= count || device >= 64) return H3_ERR_INVALID_ARG;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device) != cudaSuccess)
+    return H3_ERR_CUDA;
+  if (major != 10 || minor != 0) return H3_ERR_UNSUPPORTED;   // the kernels are built for sm_100a only
+  DeviceGuard guard;
+  if (cudaSetDevice(device) != cudaSuccess) return H3_ERR_CUDA;
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, h3::attn::attention_kernel) != cudaSuccess) return H3_ERR_UNSUPPORTED;
+  if (encode_tiled() == nullptr || device_state() == nullptr || host_pipe() == nullptr ||
+      noalloc_scratch() == nullptr)
+    return H3_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(h3::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return H3_ERR_CUDA;
+  return H3_OK;
+}
+
+void h3_shutdown(void) {
+  DeviceGuard guard;
+  release_host_pipes();
 }
 
 }  // extern "C"

@@ -33,7 +33,7 @@ def test_every_declared_symbol_is_exported():
 
 def test_struct_layouts_match_header():
     assert ctypes.sizeof(_lib.h3_segment) == 9 * 4
-    assert ctypes.sizeof(_lib.h3_rope_cfg) == 8 + 5 * 4 + 4   # double + 5 int32, padded to 8
+    assert ctypes.sizeof(_lib.h3_rope_cfg) == 8 + 6 * 4   # double + 6 int32
 
 
 def test_status_strings():
@@ -85,6 +85,8 @@ def test_rope_rejects_bad_config_and_layout():
     assert _err(h3.h3_mmrope_qk, P, P, P, P, P, 4, 1, 128, h3.rope_cfg(theta=1.0)) == h3.H3_ERR_INVALID_ARG
     assert _err(h3.h3_mmrope_qk, P, P, P, P, P, 4, 1, 128, h3.rope_cfg(pair_layout=2)) == \
         h3.H3_ERR_INVALID_ARG
+    assert _err(h3.h3_mmrope_qk, P, P, P, P, P, 4, 1, 128, h3.rope_cfg(freq_rule=2)) == \
+        h3.H3_ERR_INVALID_ARG
     assert _err(h3.h3_mmrope_qk, P, P, P, P, P, 4, 1, 256,
                 h3.rope_cfg(head_dim=256, sections=(64, 96, 96))) == h3.H3_ERR_UNSUPPORTED
     assert _err(h3.h3_mmrope_qk, P, P, P, P, P, 4, 2, 128, h3.rope_cfg()) == h3.H3_ERR_INVALID_ARG
@@ -109,3 +111,14 @@ def test_attention_rejects_bad_arguments():
     assert _err(A, P, P, P, P, 0, 1, 10, 1, 128, d_coords=P,
                 cfg=h3.rope_cfg(sections=(32, 48, 40))) == h3.H3_ERR_INVALID_ARG
     assert _err(A, P, P, P, P, 0, 1, 10, 1, 128, softmax_scale=float("nan")) == h3.H3_ERR_INVALID_ARG
+
+
+def test_init_without_a_device_fails_cleanly():
+    # no GPU in this process: an error status, nothing launched; shutdown with
+    # nothing created is a no-op
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _err(h3.h3_init, 0) in (h3.H3_ERR_CUDA, h3.H3_ERR_INVALID_ARG)
+    h3.h3_shutdown()
+    assert _lib.load().h3_version() == 101

@@ -79,20 +79,20 @@ def test_coords_reject_out_of_range_perm(h3):
 
 # ------------------------------------------------------------------- rope --
 
-def _rope_case(h3, wl, rows=None, pair_layout=0, in_place=False):
+def _rope_case(h3, wl, rows=None, pair_layout=0, in_place=False, freq_rule=0):
     perm = W.permutation(wl)
     q, k, _ = W.qkv_bf16(wl)
     coords = h3.build_coords(wl.segments, wl.n_rows, _perm_dev(perm))
     qd, kd = to_dev(q), to_dev(k)
     if in_place:
-        qo, ko = h3.mmrope_qk(qd, kd, coords, q_out=qd, k_out=kd, pair_layout=pair_layout)
+        qo, ko = h3.mmrope_qk(qd, kd, coords, q_out=qd, k_out=kd, pair_layout=pair_layout, freq_rule=freq_rule)
     else:
-        qo, ko = h3.mmrope_qk(qd, kd, coords, pair_layout=pair_layout)
+        qo, ko = h3.mmrope_qk(qd, kd, coords, pair_layout=pair_layout, freq_rule=freq_rule)
     _sync_ok(h3)
     rows = np.arange(wl.n_rows) if rows is None else rows
     num, den = ocoords.packed_coords(wl.segments, perm)
-    ang = orope.angles(ocoords.to_f64(num, den)[rows], wl.theta, wl.sections)
-    ang32 = orope.angles(ocoords.to_f32(num, den)[rows].astype(np.float64), wl.theta, wl.sections)
+    ang = orope.angles(ocoords.to_f64(num, den)[rows], wl.theta, wl.sections, freq_rule)
+    ang32 = orope.angles(ocoords.to_f32(num, den)[rows].astype(np.float64), wl.theta, wl.sections, freq_rule)
     res = []
     for x_bits, out in ((q, qo), (k, ko)):
         x = bf16_bits_to_f64(x_bits[rows])
@@ -113,6 +113,12 @@ def test_rope_half_split_and_in_place(h3):
     for frac_rne, _ in _rope_case(h3, W.workload(1), pair_layout=1):
         assert frac_rne > 0.99
     for frac_rne, _ in _rope_case(h3, W.workload(0), in_place=True):
+        assert frac_rne > 0.99
+
+
+@pytest.mark.parametrize("layout", [0, 1])
+def test_rope_single_frequency_ladder(h3, layout):
+    for frac_rne, _ in _rope_case(h3, W.workload(1), pair_layout=layout, freq_rule=1):
         assert frac_rne > 0.99
 
 
@@ -265,19 +271,20 @@ def test_pipeline_canvas_mode(h3):
 
 # -------------------------------------------------- fused RoPE on Q (a5) --
 
-@pytest.mark.parametrize("cfg,layout", [(0, 0), (1, 0), (1, 1)])
-def test_fused_q_rope_is_identical_to_rotating_first(h3, cfg, layout):
+@pytest.mark.parametrize("cfg,layout,rule", [(0, 0, 0), (1, 0, 0), (1, 1, 0), (1, 0, 1), (0, 1, 1)])
+def test_fused_q_rope_is_identical_to_rotating_first(h3, cfg, layout, rule):
     wl = W.workload(cfg)
     perm = W.permutation(wl)
     q, k, v = W.qkv_bf16(wl)
     dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
-    args = dict(perm=_perm_dev(perm), theta=wl.theta, sections=wl.sections, pair_layout=layout)
+    args = dict(perm=_perm_dev(perm), theta=wl.theta, sections=wl.sections, pair_layout=layout, freq_rule=rule)
     o_sep = h3.packed_mmrope_attention(wl.segments, dq, dk, dv, **args)
     o_fus = h3.packed_mmrope_attention(wl.segments, dq, dk, dv, fused_q_rope=True, **args)
     _sync_ok(h3)
     # same rotation arithmetic, same MMAs: bit-identical outputs
     assert torch.equal(o_sep, o_fus)
-    ref, _ = opipe.packed_mmrope_attention(wl.segments, perm, q, k, v, wl.theta, wl.sections, pair_layout=layout)
+    ref, _ = opipe.packed_mmrope_attention(wl.segments, perm, q, k, v, wl.theta, wl.sections, pair_layout=layout,
+                                           freq_rule=rule)
     check_attention(bf16_bits_to_f64(from_dev_bf16(o_fus)), ref, f"fused {wl.name}")
 
 
@@ -306,3 +313,27 @@ def test_fused_q_rope_ragged_batch(h3):
     o_fus = h3.packed_attention(dq, kr, dv, coords=coords)
     _sync_ok(h3)
     assert torch.equal(o_sep, o_fus)
+
+
+# -------------------------------------------------------------- lifecycle --
+
+def test_init_and_shutdown(h3):
+    dev = torch.cuda.current_device()
+    h3.h3_init(dev)
+    h3.h3_init(dev)                                   # again: harmless
+    with pytest.raises(h3.H3Error) as e:
+        h3.h3_init(torch.cuda.device_count())
+    assert e.value.status == h3.H3_ERR_INVALID_ARG
+    assert torch.cuda.current_device() == dev
+    # the host-buffer path works, is torn down, and works again after shutdown
+    wl = W.workload(0)
+    q, k, v = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) for a in W.qkv_bf16(wl))
+    perm = torch.from_numpy(W.permutation(wl).astype(np.int32))
+    o1 = h3.packed_mmrope_attention_host(wl.segments, q, k, v, perm=perm)
+    torch.cuda.synchronize()
+    h3.h3_shutdown()
+    o2 = h3.packed_mmrope_attention_host(wl.segments, q, k, v, perm=perm)
+    torch.cuda.synchronize()
+    _sync_ok(h3)
+    assert torch.equal(o1, o2)
+    assert torch.cuda.current_device() == dev
