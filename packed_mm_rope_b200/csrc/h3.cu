@@ -41,13 +41,8 @@ const DeviceState* device_state() {
   std::lock_guard<std::mutex> lock(mu);
   DeviceState& st = states[dev];
   if (!st.ready) {
-    size_t adaln_most = 0;
-    for (int hdn = 8; hdn <= h3::ADALN_MAX_HIDDEN; hdn += 8)
-      adaln_most = std::max(adaln_most, h3::adaln_smem_bytes(hdn));
     if (cudaFuncSetAttribute(h3::attn::attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(h3::attn::SMEM_BYTES)) != cudaSuccess ||
-        cudaFuncSetAttribute(h3::adaln_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(adaln_most)) != cudaSuccess)
+                             static_cast<int>(h3::attn::SMEM_BYTES)) != cudaSuccess)
       return nullptr;
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) st.sms = n;
@@ -283,15 +278,13 @@ h3_status h3_adaln_modulate(const void* d_x, void* d_y, const int32_t* d_timeste
   if (!d_x || !d_y || !d_timestep_index || !d_token_tag || !d_table) return H3_ERR_INVALID_ARG;
   if (x_row_stride % 8 || y_row_stride % 8 || !aligned16(d_x) || !aligned16(d_y) || !aligned16(d_table))
     return H3_ERR_UNSUPPORTED;
-  const size_t smem = h3::adaln_smem_bytes(hidden);
-  if (device_state() == nullptr) return H3_ERR_CUDA;
-  // one CTA per SM (the rings fill shared memory); contiguous row blocks
-  const long long grid = std::min<long long>(sm_count(), (n_rows + h3::ADALN_WARPS - 1) / h3::ADALN_WARPS);
-  const long long per_cta = (n_rows + grid - 1) / grid;
-  h3::adaln_kernel<<<static_cast<int>(grid), h3::ADALN_THREADS, smem, as_stream(stream)>>>(
+  // one resident wave: ADALN_CTAS_PER_SM CTAs per SM, rows grid-strided over the row groups
+  const long long grid = std::min<long long>(static_cast<long long>(h3::ADALN_CTAS_PER_SM) * sm_count(),
+                                             (n_rows + h3::ADALN_GROUPS - 1) / h3::ADALN_GROUPS);
+  h3::adaln_kernel<<<static_cast<int>(grid), h3::ADALN_THREADS, 0, as_stream(stream)>>>(
       static_cast<const uint4*>(d_x), static_cast<uint4*>(d_y), d_timestep_index, d_token_tag,
       reinterpret_cast<const float4*>(d_table), n_entries, n_rows, hidden / 8, x_row_stride / 8, y_row_stride / 8,
-      eps, g_wait_limit_ns, per_cta);
+      eps);
   return cudaGetLastError() == cudaSuccess ? H3_OK : H3_ERR_CUDA;
 }
 
