@@ -204,8 +204,10 @@ h3_status h3_mmrope_qk(const void* d_q, const void* d_k, void* d_q_out, void* d_
     return H3_ERR_UNSUPPORTED;
   if (static_cast<long long>(n_heads) * 16 > (1ll << 30)) return H3_ERR_INVALID_ARG;
   const h3::RopeTable tab = make_rope_table(cfg);
-  const long long nblk = (n_rows + h3::ROPE_ROWS - 1) / h3::ROPE_ROWS;
-  const long long cap = 8LL * sm_count();
+  // one warp per row; four CTAs per SM queued for two resident (tail balance)
+  const long long warps_per_cta = h3::ROPE_THREADS / 32;
+  const long long nblk = (n_rows + warps_per_cta - 1) / warps_per_cta;
+  const long long cap = 2LL * h3::ROPE_CTAS_PER_SM * sm_count();
   const int grid = static_cast<int>(nblk < cap ? nblk : cap);
   const long long stride16 = row_stride / 8;
   auto q = static_cast<const uint4*>(d_q);

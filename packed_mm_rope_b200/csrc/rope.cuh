@@ -5,12 +5,11 @@
 // page traces position_ids[:, 0] (t) into rope() and the rotation of Q and K,
 // with inverse frequencies computed from rope_theta / rope_freq_dim.
 //
-// HBM-bound streaming kernel.  A CTA owns ROWS packed rows at a time: it
-// first builds the 64 (cos, sin) pairs of each row in shared memory (fp64
-// angle = fp64 coordinate x fp64 inverse frequency, fp64 sincos, rounded to
-// fp32), then streams both tensors with 16-byte loads.  The angles of a row
-// are shared by all heads and by Q and K, so the trigonometry is paid once
-// per row, not per element.  Persistent grid, grid-stride over row blocks.
+// HBM-bound streaming kernel: one warp per packed row streams both tensors
+// with 16-byte loads.  The (cos, sin) of a rotary pair (fp64 angle = fp64
+// coordinate x fp64 inverse frequency, fp64 sincos, rounded to fp32) is shared
+// by all heads and by Q and K, so each lane computes the few pairs it meets
+// once per row, not per element.  Persistent grid, grid-stride over rows.
 #pragma once
 
 #include "common.cuh"
@@ -23,8 +22,7 @@ struct RopeTable {
 };
 
 constexpr int ROPE_THREADS = 256;
-constexpr int ROPE_ROWS = 8;      // rows per block iteration
-constexpr int ROPE_UNROLL = 4;    // independent 16-byte chunks in flight per thread
+constexpr int ROPE_CTAS_PER_SM = 2;   // register-limited residency of rope_kernel
 
 // (cos, sin) of pair p for a row with coordinates crd[0..2]: fp64 angle =
 // fp64(coordinate) x fp64 inverse frequency, fp64 sincos, each rounded to fp32.
@@ -75,67 +73,67 @@ __device__ __forceinline__ void rotate_half(uint4& a, uint4& b, const float2* cs
   b = make_uint4(wb[0], wb[1], wb[2], wb[3]);
 }
 
-// q / qo may both be null: then only K is rotated.
-// LAYOUT 0: pair p = dims (2p, 2p+1); one work item = one 16-byte chunk.
-// LAYOUT 1: pair p = dims (p, p+64);  one work item = chunks c and c+8 of a head.
+// One warp per packed row.  A row of one tensor is n_heads x 16 chunks of 16
+// bytes; lane l handles the chunks (or, half-split, the chunk pairs) l, l + 32,
+// ...  Because 32 is a multiple of the chunks per head, a lane always meets the
+// same rotary pairs (4 adjacent pairs, or 8 half-split pairs) in every head, so
+// it computes their (cos, sin) itself, once per row, while its first loads are
+// in flight: no shared memory and no block barrier.  q / qo may both be null:
+// then only K is rotated.  LAYOUT 0: pair p = dims (2p, 2p+1), one item = one
+// chunk; LAYOUT 1: pair p = dims (p, p+64), one item = chunks c and c+8.
 template <int LAYOUT>
-__global__ void __launch_bounds__(ROPE_THREADS) rope_kernel(
+__global__ void __launch_bounds__(ROPE_THREADS, ROPE_CTAS_PER_SM) rope_kernel(
     const uint4* q, const uint4* k, uint4* qo, uint4* ko, const float* __restrict__ coords,
     long long n_rows, int n_heads, long long stride16, const RopeTable tab) {
-  __shared__ float2 cs[ROPE_ROWS][64];
-  constexpr int ITEMS_PER_HEAD = LAYOUT == 0 ? 16 : 8;
-  const int items_per_row = n_heads * ITEMS_PER_HEAD;
-  const long long nblk = (n_rows + ROPE_ROWS - 1) / ROPE_ROWS;
-
-  for (long long blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
-    const long long r0 = blk * ROPE_ROWS;
-    const int nr = static_cast<int>(min(static_cast<long long>(ROPE_ROWS), n_rows - r0));
-    __syncthreads();   // previous block's readers are done with cs
-    for (int i = threadIdx.x; i < nr * 64; i += ROPE_THREADS) {
-      const int r = i >> 6, p = i & 63;
-      cs[r][p] = rope_cos_sin(tab, coords + 3 * (r0 + r), p);
-    }
-    __syncthreads();
-
-    const int total = nr * items_per_row;
-    for (int base = threadIdx.x; base < total; base += ROPE_THREADS * ROPE_UNROLL) {
-      uint4 qa[ROPE_UNROLL], ka[ROPE_UNROLL], qb[ROPE_UNROLL], kb[ROPE_UNROLL];
-      long long off[ROPE_UNROLL];
-      int pair0[ROPE_UNROLL], row[ROPE_UNROLL];
+  constexpr int IPH = LAYOUT == 0 ? 16 : 8;        // work items per head
+  constexpr int PPI = LAYOUT == 0 ? 4 : 8;         // rotary pairs per item
+  constexpr int B = LAYOUT == 0 ? 7 : 4;           // items per lane in flight
+  const int lane = threadIdx.x & 31;
+  const int sub = lane % IPH;                      // item index within the head
+  const long long gw = (static_cast<long long>(blockIdx.x) * ROPE_THREADS + threadIdx.x) >> 5;
+  const long long nw = (static_cast<long long>(gridDim.x) * ROPE_THREADS) >> 5;
+  const int items = n_heads * IPH;
+  const bool has_q = q != nullptr;
+  for (long long r = gw; r < n_rows; r += nw) {
+    const long long row_off = r * stride16;
+    float2 cs[PPI];
+    bool first = true;
+    for (int i0 = lane; i0 < items; i0 += 32 * B) {
+      uint4 qa[B], ka[B], qb[B], kb[B];
+      long long off[B];
 #pragma unroll
-      for (int u = 0; u < ROPE_UNROLL; ++u) {
-        const int item = base + u * ROPE_THREADS;
+      for (int u = 0; u < B; ++u) {
+        const int item = i0 + 32 * u;
         off[u] = -1;
-        if (item < total) {
-          const int r = item / items_per_row;
-          const int c = item - r * items_per_row;
-          const int head = c / ITEMS_PER_HEAD;
-          const int sub = c - head * ITEMS_PER_HEAD;
-          row[u] = r;
-          off[u] = (r0 + r) * stride16 + head * 16 + sub;
-          pair0[u] = LAYOUT == 0 ? 4 * sub : 8 * sub;
-          if (q != nullptr) qa[u] = __ldcs(q + off[u]);
+        if (item < items) {
+          off[u] = row_off + (item / IPH) * 16 + sub;
+          if (has_q) qa[u] = __ldcs(q + off[u]);
           ka[u] = __ldcs(k + off[u]);
           if (LAYOUT == 1) {
-            if (q != nullptr) qb[u] = __ldcs(q + off[u] + 8);
+            if (has_q) qb[u] = __ldcs(q + off[u] + 8);
             kb[u] = __ldcs(k + off[u] + 8);
           }
         }
       }
+      if (first) {
+        const float* crd = coords + 3 * r;
 #pragma unroll
-      for (int u = 0; u < ROPE_UNROLL; ++u) {
+        for (int m = 0; m < PPI; ++m) cs[m] = rope_cos_sin(tab, crd, PPI * sub + m);
+        first = false;
+      }
+#pragma unroll
+      for (int u = 0; u < B; ++u) {
         if (off[u] < 0) continue;
-        const float2* c = &cs[row[u]][pair0[u]];
         if (LAYOUT == 0) {
-          if (q != nullptr) __stcs(qo + off[u], rotate_adjacent(qa[u], c));
-          __stcs(ko + off[u], rotate_adjacent(ka[u], c));
+          if (has_q) __stcs(qo + off[u], rotate_adjacent(qa[u], cs));
+          __stcs(ko + off[u], rotate_adjacent(ka[u], cs));
         } else {
-          if (q != nullptr) {
-            rotate_half(qa[u], qb[u], c);
+          if (has_q) {
+            rotate_half(qa[u], qb[u], cs);
             __stcs(qo + off[u], qa[u]);
             __stcs(qo + off[u] + 8, qb[u]);
           }
-          rotate_half(ka[u], kb[u], c);
+          rotate_half(ka[u], kb[u], cs);
           __stcs(ko + off[u], ka[u]);
           __stcs(ko + off[u] + 8, kb[u]);
         }
