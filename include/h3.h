@@ -344,7 +344,10 @@ h3_status h3_packed_mmrope_attention_host_noalloc(const h3_segment* segs, int32_
                                                   void* stream);
 
 /*
- * Synchronise `stream`, then read and clear this device's error word.
+ * Read and clear this device's error word (one word per device, shared by
+ * all streams) in one atomic step ordered after the work already queued on
+ * `stream`, then synchronise `stream`.  A fault raised by a kernel still
+ * running on another stream is reported by a later call.
  * Returns H3_OK, H3_ERR_TIMEOUT, H3_ERR_DEVICE_INPUT or H3_ERR_CUDA.
  */
 h3_status h3_check_device_error(void* stream);

@@ -21,6 +21,12 @@ enum : unsigned int {
 };
 
 __device__ unsigned int g_error_word;
+__device__ unsigned int g_error_snapshot;   // last value taken by take_error_word
+
+// Read and clear the error word in one atomic step, so that a bit raised by a
+// kernel running concurrently on another stream is never lost between the
+// read and the clear.
+__global__ void take_error_word() { g_error_snapshot = atomicExch(&g_error_word, 0u); }
 
 // ------------------------------------------------------------ timing ----
 

@@ -4,6 +4,7 @@
 // The library allocates no device memory; the per-device error word is a
 // static __device__ variable of this module.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -19,7 +20,7 @@ namespace {
 
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;   // 2 s per wait
 constexpr uint64_t kDrainLimitNs = 2000000000ull;
-uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
+std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -137,7 +138,7 @@ const char* h3_status_str(int32_t status) {
 int32_t h3_version(void) { return 101; }
 
 h3_status h3_set_wait_limit_ns(uint64_t ns) {
-  g_wait_limit_ns = ns == 0 ? kDefaultWaitLimitNs : ns;
+  g_wait_limit_ns.store(ns == 0 ? kDefaultWaitLimitNs : ns);
   return H3_OK;
 }
 
@@ -257,7 +258,7 @@ h3_status h3_packed_attention(const void* d_q, const void* d_k, const void* d_v,
   p.o_row_stride = row_stride;
   p.o_batch_stride = row_stride * n_rows;
   p.lse = d_lse;
-  p.wait_limit_ns = g_wait_limit_ns;
+  p.wait_limit_ns = g_wait_limit_ns.load();
   p.drain_limit_ns = kDrainLimitNs;
   p.coords = d_coords;
   p.rope_layout = d_coords ? cfg->pair_layout : 0;
@@ -520,11 +521,12 @@ h3_status h3_packed_mmrope_attention_host_noalloc(const h3_segment* segs, int32_
 }
 
 h3_status h3_check_device_error(void* stream) {
-  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return H3_ERR_CUDA;
-  unsigned int word = 0, zero = 0;
-  if (cudaMemcpyFromSymbol(&word, h3::g_error_word, sizeof(word)) != cudaSuccess) return H3_ERR_CUDA;
-  if (word != 0 && cudaMemcpyToSymbol(h3::g_error_word, &zero, sizeof(zero)) != cudaSuccess)
+  // ordered after the work already on `stream`
+  h3::take_error_word<<<1, 1, 0, as_stream(stream)>>>();
+  if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(as_stream(stream)) != cudaSuccess)
     return H3_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, h3::g_error_snapshot, sizeof(word)) != cudaSuccess) return H3_ERR_CUDA;
   if (word & h3::DEVERR_TIMEOUT) return H3_ERR_TIMEOUT;
   if (word & h3::DEVERR_INPUT) return H3_ERR_DEVICE_INPUT;
   return H3_OK;
