@@ -88,9 +88,6 @@ constexpr uint32_t TMEM_S0 = 0, TMEM_O0 = 256;
 #define H3_EXP2_FMA_EVERY 0   // measured slower at every share on B200
 #endif
 constexpr int EXP2_FMA_EVERY = H3_EXP2_FMA_EVERY;
-#ifndef H3_EXP_F16X2
-#define H3_EXP_F16X2 0
-#endif
 
 // 2^x on the FMA pipe: x = n + f with n = nearest integer (the 1.5 * 2^23
 // rounding trick), 2^f by a degree-3 polynomial whose coefficients minimise the
