@@ -63,3 +63,32 @@ def test_adaln_in_place_and_bad_index(h3):
     keep = np.delete(np.arange(n), 7)
     ref = oadaln.adaln_modulate(bf16_bits_to_f64(x)[keep], ts[keep], tags[keep], table.astype(np.float64))
     assert (np.abs(got[keep] - ref) <= bf16_ulp(ref) + 1e-5 * (1 + np.abs(ref))).all()
+
+
+@pytest.mark.parametrize("n,hidden", [(1, 8), (3, 1032), (257, 8192), (130, 4104)])
+def test_adaln_widths_and_ragged_row_counts(h3, n, hidden):
+    # widths at the chunk boundaries of the kernel (one 16-byte chunk; 129 chunks,
+    # one past a whole 128-thread pass; the 8,192 maximum; 513 chunks) and row
+    # counts that leave the last row group of a CTA half-used
+    x = W.normal_bf16(77 + n, 0, (n, hidden), scale=3.0)
+    rng = np.random.default_rng(n)
+    ts = rng.integers(0, 2, n).astype(np.int32)
+    tags = rng.integers(0, 3, n).astype(np.int32)
+    table = (rng.standard_normal((6, 2, hidden)) * 0.3).astype(np.float32)
+    y = h3.adaln_modulate(to_dev(x), torch.from_numpy(ts).cuda(), torch.from_numpy(tags).cuda(),
+                          torch.from_numpy(table).cuda(), eps=1e-5)
+    assert h3.h3_check_device_error() == h3.H3_OK
+    got = bf16_bits_to_f64(from_dev_bf16(y))
+    ref = oadaln.adaln_modulate(bf16_bits_to_f64(x), ts, tags, table.astype(np.float64), eps=1e-5)
+    err = np.abs(got - ref)
+    bound = bf16_ulp(ref) + 1e-5 * (1.0 + np.abs(ref))
+    assert (err <= bound).all(), (err.max(), (err > bound).sum())
+
+
+def test_adaln_rejects_unsupported_widths(h3):
+    x = torch.zeros((2, 8200), dtype=torch.bfloat16, device="cuda")
+    idx = torch.zeros(2, dtype=torch.int32, device="cuda")
+    table = torch.zeros((3, 2, 8200), dtype=torch.float32, device="cuda")
+    with pytest.raises(h3.H3Error) as e:
+        h3.adaln_modulate(x, idx, idx, table)
+    assert e.value.status == h3.H3_ERR_UNSUPPORTED

@@ -337,3 +337,23 @@ def test_init_and_shutdown(h3):
     _sync_ok(h3)
     assert torch.equal(o1, o2)
     assert torch.cuda.current_device() == dev
+
+
+@pytest.mark.parametrize("heads,layout", [(1, 0), (3, 0), (5, 1), (64, 0), (2, 1)])
+def test_rope_head_counts(h3, heads, layout):
+    # one warp per row, lane l on chunks l, l + 32, ...: head counts that leave
+    # lanes idle (1 head = 16 chunks), odd counts, and a wide row
+    wl = W.workload(0)
+    perm = W.permutation(wl)
+    q, k = (W.normal_bf16(500 + heads + i, 0, (wl.n_rows, heads, 128)) for i in range(2))
+    coords = h3.build_coords(wl.segments, wl.n_rows, _perm_dev(perm))
+    qo, ko = h3.mmrope_qk(to_dev(q), to_dev(k), coords, pair_layout=layout)
+    _sync_ok(h3)
+    num, den = ocoords.packed_coords(wl.segments, perm)
+    ang = orope.angles(ocoords.to_f64(num, den), wl.theta, wl.sections)
+    ang32 = orope.angles(ocoords.to_f32(num, den).astype(np.float64), wl.theta, wl.sections)
+    for x_bits, out in ((q, qo), (k, ko)):
+        x = bf16_bits_to_f64(x_bits)
+        frac_rne, _ = check_rope(from_dev_bf16(out), orope.rotate(x, ang, layout), x, layout,
+                                 dang=np.abs(ang32 - ang))
+        assert frac_rne > 0.99
