@@ -8,7 +8,6 @@ and their V are computed once, and each later step rotates and writes only
 the fresh rows (a row-range view of the same buffers) before attending over
 all rows.  The result must equal recomputing every row.
 """
-import numpy as np
 import pytest
 
 torch = pytest.importorskip("torch")

@@ -4,7 +4,6 @@ attention kernel is bounded by device global time.  With the limit forced to
 memory and returns; the host reads H3_ERR_TIMEOUT from the error word, and the
 next call on the same context computes correct results again.
 """
-import numpy as np
 import pytest
 
 torch = pytest.importorskip("torch")
