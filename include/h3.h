@@ -29,10 +29,15 @@
  *     NULL = the legacy default stream).  Arguments are validated on the host
  *     before anything is launched; a call that returns an error launched
  *     nothing, except H3_ERR_CUDA reported by the launch itself.
- *   - The library allocates no device memory.  Kernel-side faults in the
- *     inputs (a permutation entry out of range, a bounded wait that expired)
- *     are recorded in a per-device error word; h3_check_device_error reads
- *     and clears it.
+ *   - The library allocates no device memory at run time.  Its only device
+ *     storage is static module data, held by every GPU that loads the
+ *     library until the process exits: 2 KB of error words and the fixed
+ *     H3_NOALLOC_SCRATCH_BYTES (64 MiB) scratch array of
+ *     h3_packed_mmrope_attention_host_noalloc.
+ *   - Kernel-side faults in the inputs (a permutation entry out of range, a
+ *     bounded wait that expired) are recorded in an error word of the stream
+ *     the kernel ran on; h3_check_device_error(stream) reads and clears it.
+ *   - Host calls are thread-safe for distinct streams.
  *   - Q/K/V/O tensors are bf16 in row-major [batch][n_rows][n_heads][head_dim]
  *     with a row stride of `row_stride` elements (>= n_heads * head_dim,
  *     a multiple of 8) and a batch stride of n_rows * row_stride elements.
@@ -144,9 +149,11 @@ int32_t h3_version(void);
  * kernels load on it, then does once what every other call otherwise does
  * lazily on first use: the shared-memory opt-ins of the kernels, the lookup of
  * the driver's tensor-map encoder, the host-buffer pipeline's two streams and
- * events, the address of the no-allocation scratch; and clears the device
- * error word.  Allocates no device memory.  The calling thread's current
- * device is left as it was.  Calling it again is harmless.
+ * events, the address of the no-allocation scratch; and clears the device's
+ * error words.  Allocates no device memory at run time (loading the kernels
+ * on the device commits the module's static arrays, among them the 64 MiB
+ * no-allocation scratch).  The calling thread's current device is left as it
+ * was.  Calling it again is harmless.
  * Errors: H3_ERR_INVALID_ARG (no such device), H3_ERR_UNSUPPORTED (another
  * architecture, or the kernels do not load), H3_ERR_CUDA.
  */
@@ -154,10 +161,13 @@ h3_status h3_init(int32_t device);
 
 /*
  * h3_shutdown -- releases what the library created: on every device, waits
- * for and destroys the host-buffer pipeline's streams and events.  Must not
- * run concurrently with another call of the library.  The library stays
- * usable: a later call re-creates what it needs.  The calling thread's
- * current device is left as it was.
+ * for and destroys the host-buffer pipeline's streams and events, and forgets
+ * every per-device lookup (kernel attributes, the scratch array's address,
+ * the stream-to-error-word map).  Must not run concurrently with another
+ * call of the library.  The library stays usable: a later call re-creates
+ * what it needs.  Call it before cudaDeviceReset (a reset replaces the
+ * module's arrays and attributes, so cached lookups would be stale).  The
+ * calling thread's current device is left as it was.
  */
 void h3_shutdown(void);
 
@@ -297,7 +307,11 @@ uint64_t h3_host_workspace_bytes(int64_t n_rows, int32_t n_heads);
  *                     to wait for h_o.  Host buffers must stay valid until then.
  * Errors: as the three calls it composes; H3_ERR_INVALID_ARG for a NULL or
  * misaligned workspace; H3_ERR_CUDA if an internal stream or event cannot be
- * created (they are created once per device and kept until process exit).
+ * created (they are created once per device and kept until h3_shutdown).
+ * Every argument, the segment table included, is checked before anything is
+ * queued.  If a CUDA call fails after copies were queued, `stream` is still
+ * ordered after every queued copy before the error is returned, so
+ * synchronising `stream` makes the host buffers safe to release.
  */
 h3_status h3_packed_mmrope_attention_host(const h3_segment* segs, int32_t nseg, const int32_t* h_perm,
                                           const void* h_q, const void* h_k, const void* h_v, void* h_o,
@@ -331,7 +345,9 @@ h3_status h3_packed_mmrope_attention_host(const h3_segment* segs, int32_t nseg, 
  *                  is queued (about 65k row-heads: e.g. 4,584 rows x 8 heads)
  *   first call     the first call on each device looks up the scratch
  *                  array's device address (cudaGetSymbolAddress) and caches
- *                  it; make that first call before any stream capture
+ *                  it until h3_shutdown (h3_init does the same up front);
+ *                  make that first call before any stream capture, and call
+ *                  h3_shutdown before a cudaDeviceReset
  *   sharing        every call on a device uses the same scratch and leaves its
  *                  contents behind; nothing in it has to start at zero (each
  *                  call writes every byte it later reads).  Calls whose GPU
@@ -344,10 +360,13 @@ h3_status h3_packed_mmrope_attention_host_noalloc(const h3_segment* segs, int32_
                                                   void* stream);
 
 /*
- * Read and clear this device's error word (one word per device, shared by
- * all streams) in one atomic step ordered after the work already queued on
- * `stream`, then synchronise `stream`.  A fault raised by a kernel still
- * running on another stream is reported by a later call.
+ * Read and clear the error word of `stream` on the current device in one
+ * atomic step ordered after the work already queued on `stream`, then
+ * synchronise `stream`.  Every kernel the library launches records its faults
+ * in the word of the stream it was launched on, so a check reports only that
+ * stream's faults: distinct streams may be checked from distinct threads.
+ * The library keeps 255 such words per device, handed out to streams in the
+ * order it first sees them; streams beyond the 255th share one further word.
  * Returns H3_OK, H3_ERR_TIMEOUT, H3_ERR_DEVICE_INPUT or H3_ERR_CUDA.
  */
 h3_status h3_check_device_error(void* stream);

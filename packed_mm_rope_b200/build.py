@@ -8,6 +8,7 @@ at run time, so no libcuda link is needed.
 """
 from __future__ import annotations
 
+import glob
 import os
 import shutil
 import subprocess
@@ -16,8 +17,14 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libh3.so")
-SOURCES = [os.path.join(HERE, "csrc", f) for f in ("h3.cu", "common.cuh", "coords.cuh", "rope.cuh", "attention.cuh")]
+CSRC = os.path.join(HERE, "csrc")
 HEADER = os.path.join(ROOT, "include", "h3.h")
+
+
+def sources() -> list:
+    """Every file the library is built from: all of csrc/ and the public header."""
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))) + [HEADER]
+
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -38,16 +45,14 @@ def up_to_date() -> bool:
     if not os.path.exists(LIB):
         return False
     t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(s) <= t for s in SOURCES + [HEADER, __file__])
+    return all(os.path.getmtime(s) <= t for s in sources() + [__file__])
 
 
 def build_library(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
-    # H3_NVCC_DEFINES="-DNAME=VALUE ..." passes tuning macros (e.g. H3_EXP2_FMA_EVERY)
-    extra = os.environ.get("H3_NVCC_DEFINES", "").split()
-    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"),
-           os.path.join(HERE, "csrc", "h3.cu"), "-o", LIB + ".tmp"]
+    cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"),
+           os.path.join(CSRC, "h3.cu"), "-o", LIB + ".tmp"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)

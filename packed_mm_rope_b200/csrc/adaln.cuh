@@ -48,7 +48,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 __global__ void __launch_bounds__(ADALN_THREADS, ADALN_CTAS_PER_SM) adaln_kernel(
     const uint4* x, uint4* y, const int32_t* __restrict__ ts_idx, const int32_t* __restrict__ tags,
     const float4* __restrict__ table, int n_entries, long long n_rows, int chunks, long long x_stride16,
-    long long y_stride16, float eps) {
+    long long y_stride16, float eps, int err_slot) {
   __shared__ float2 partial[ADALN_GROUPS][2][ADALN_WARPS_PER_GROUP];   // (S1, S2) per warp
   const int g = threadIdx.x / ADALN_GROUP;
   const int t = threadIdx.x % ADALN_GROUP;
@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(ADALN_THREADS, ADALN_CTAS_PER_SM) adaln_kernel
     const float rstd = rsqrtf(var + eps);
     const long long e = static_cast<long long>(ts_idx[r]) * 3 + tags[r];
     const bool bad = e < 0 || e >= n_entries;
-    if (bad && t == 0) atomicOr(&g_error_word, DEVERR_INPUT);
+    if (bad && t == 0) raise_error(err_slot, DEVERR_INPUT);
     const float4* ent = table + (bad ? 0 : e) * 4LL * chunks;
     // y = x * a + b with a = rstd * (1 + scale), b = shift - mean * a
     const float2 rs2 = make_float2(rstd, rstd), nm2 = make_float2(-mean, -mean), one2 = make_float2(1.f, 1.f);

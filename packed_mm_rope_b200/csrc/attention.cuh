@@ -55,10 +55,7 @@ namespace attn {
 constexpr int BM = 128;          // query rows per tile (MMA M)
 constexpr int BN = 128;          // key rows per tile  (S MMA N, PV MMA K)
 constexpr int HD = 128;          // head dim
-#ifndef H3_KV_STAGES
-#define H3_KV_STAGES 4
-#endif
-constexpr int KV_STAGES = H3_KV_STAGES;
+constexpr int KV_STAGES = 4;     // K/V ring slots of 32 KB
 constexpr int THREADS = 320;
 constexpr uint32_t TILE_BYTES = BM * HD * 2;     // 32768
 constexpr uint32_t HALF_BYTES = TILE_BYTES / 2;  // 16384
@@ -80,61 +77,18 @@ constexpr uint32_t IDESC_O = idesc_bf16_f32(BM, HD, false, true);    // P from T
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_S0 = 0, TMEM_O0 = 256;
 
-// Every EXP2_FMA_EVERY-th pair of exponentials is computed on the FMA pipe
-// (0 = all on the MUFU unit).  The MUFU unit issues 16 exponentials per clock
-// per SM, the same time the tensor core needs for a 128 x 128 x 128 tile pair,
-// so moving a share of them to the FMA pipe takes the unit off the critical path.
-#ifndef H3_EXP2_FMA_EVERY
-#define H3_EXP2_FMA_EVERY 0   // measured slower at every share on B200
-#endif
-constexpr int EXP2_FMA_EVERY = H3_EXP2_FMA_EVERY;
-
-// 2^x on the FMA pipe: x = n + f with n = nearest integer (the 1.5 * 2^23
-// rounding trick), 2^f by a degree-3 polynomial whose coefficients minimise the
-// maximum RELATIVE error on [-1/2, 1/2] (Remez exchange; fit_exp2_poly.py
-// regenerates them; max relative error 7.5e-5, below bf16's 2^-9 rounding of
-// P), and 2^n added to the exponent field.  x is clamped below at -126 so the
-// exponent stays in range; values that small are zero at bf16 resolution.
-constexpr float EXP2_C0 = 0.9999280571937561f;
-constexpr float EXP2_C1 = 0.6932609677314758f;
-constexpr float EXP2_C2 = 0.2426111251115799f;
-constexpr float EXP2_C3 = 0.0551716685295105f;
-
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -126.f);
-  const float j = __fadd_rn(x, 12582912.f);      // 1.5 * 2^23 + round(x)
-  const float f = __fsub_rn(x, __fsub_rn(j, 12582912.f));
-  float p = fmaf(EXP2_C3, f, EXP2_C2);
-  p = fmaf(p, f, EXP2_C1);
-  p = fmaf(p, f, EXP2_C0);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(j) << 23));
-}
-
 // Waits of the single MMA-issuing thread spin with test_wait (never suspend):
 // it is on the critical path of both query tiles.
 __device__ __forceinline__ bool mma_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
-                                         uint64_t limit) {
-  return mbar_spin_bounded(bar, parity, abort, limit);
-}
-
-// exp2_fma for two values with packed fp32x2 arithmetic (same steps).
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-  const float2 big = make_float2(12582912.f, 12582912.f);
-  x = make_float2(fmaxf(x.x, -126.f), fmaxf(x.y, -126.f));
-  const float2 j = __fadd2_rn(x, big);
-  const float2 f = __ffma2_rn(__fadd2_rn(j, make_float2(-12582912.f, -12582912.f)), make_float2(-1.f, -1.f), x);
-  float2 q = __ffma2_rn(make_float2(EXP2_C3, EXP2_C3), f, make_float2(EXP2_C2, EXP2_C2));
-  q = __ffma2_rn(q, f, make_float2(EXP2_C1, EXP2_C1));
-  q = __ffma2_rn(q, f, make_float2(EXP2_C0, EXP2_C0));
-  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(j.x) << 23)),
-                     __int_as_float(__float_as_int(q.y) + (__float_as_int(j.y) << 23)));
+                                         uint64_t limit, int err_slot) {
+  return mbar_spin_bounded(bar, parity, abort, limit, err_slot);
 }
 
 // All lanes wait; the warp proceeds only if every lane saw the phase complete,
 // so the .sync.aligned tcgen05 instructions that follow run converged.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
-                                          uint64_t limit) {
-  const bool r = mbar_wait_bounded(bar, parity, abort, limit);
+                                          uint64_t limit, int err_slot) {
+  const bool r = mbar_wait_bounded(bar, parity, abort, limit, err_slot);
   return __all_sync(0xffffffffu, r);
 }
 
@@ -149,6 +103,7 @@ struct Params {
   float* lse;                     // [B][H][N] or null
   unsigned long long wait_limit_ns;
   unsigned long long drain_limit_ns;
+  int err_slot;                   // error word of the launching stream
   // fused RoPE on Q (coords == null: Q arrives rotated)
   const float* coords;            // [B][N][3]
   int rope_layout;                // 0 adjacent pairs, 1 half-split
@@ -167,15 +122,7 @@ __device__ __forceinline__ void exp_half(const float (&x)[64], float sl2, float 
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
     const float2 y = __ffma2_rn(make_float2(x[2 * c], x[2 * c + 1]), c2, mm);
-    float p0, p1;
-    if (EXP2_FMA_EVERY > 0 && (c % (EXP2_FMA_EVERY > 0 ? EXP2_FMA_EVERY : 1)) == EXP2_FMA_EVERY - 1) {
-      const float2 e = exp2_fma2(y);
-      p0 = e.x;
-      p1 = e.y;
-    } else {
-      p0 = ex2_approx(y.x);
-      p1 = ex2_approx(y.y);
-    }
+    const float p0 = ex2_approx(y.x), p1 = ex2_approx(y.y);
     acc[c & 3] = __fadd2_rn(acc[c & 3], make_float2(p0, p1));
     pk[c] = pack_bf16x2(p0, p1);
   }
@@ -222,6 +169,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int q_row0 = blockIdx.x * (2 * BM);
   const int nkv = p.n_kv_tiles;
   const uint64_t limit = p.wait_limit_ns;
+  const int eslot = p.err_slot;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -270,7 +218,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       for (int idx = 0; idx < 2 * nkv; ++idx) {
         const int s = idx % KV_STAGES;
         const int use = idx / KV_STAGES;
-        if (use > 0 && !mbar_wait_bounded(bar_kv_empty(s), (use - 1) & 1, abort_flag, limit)) break;
+        if (use > 0 && !mbar_wait_bounded(bar_kv_empty(s), (use - 1) & 1, abort_flag, limit, eslot)) break;
         const CUtensorMap* tm = (idx & 1) ? &tm_v : &tm_k;
         const int row = (idx >> 1) * BN;
         const uint32_t dst = base + SMEM_KV + s * TILE_BYTES;
@@ -282,10 +230,10 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       // Drain: every load this thread started must land before the CTA exits.
       // The drain ignores the abort flag (a never-raised local flag).
       volatile uint32_t never = 0u;
-      for (int i = 0; i < 2; ++i) mbar_wait_bounded(bar_q_full(i), 0, &never, p.drain_limit_ns);
+      for (int i = 0; i < 2; ++i) mbar_wait_bounded(bar_q_full(i), 0, &never, p.drain_limit_ns, eslot);
       for (int idx = (issued > KV_STAGES ? issued - KV_STAGES : 0); idx < issued; ++idx)
         mbar_wait_bounded(bar_kv_full(idx % KV_STAGES), (idx / KV_STAGES) & 1, &never,
-                          p.drain_limit_ns);
+                          p.drain_limit_ns, eslot);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA ----
@@ -316,24 +264,24 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       };
       // P_i(j) in two halves; the first half's completion is announced on pva_done
       auto issue_pv_tile = [&](int i, int vs, int j) -> bool {
-        if (!mma_wait(bar_p_full(i, 0), j & 1, abort_flag, limit)) return false;
+        if (!mma_wait(bar_p_full(i, 0), j & 1, abort_flag, limit, eslot)) return false;
         tc_fence_after();
         issue_pv(i, vs, 0, j > 0);
         tc_commit(bar_pva_done(i));
-        if (!mma_wait(bar_p_full(i, 1), j & 1, abort_flag, limit)) return false;
+        if (!mma_wait(bar_p_full(i, 1), j & 1, abort_flag, limit, eslot)) return false;
         tc_fence_after();
         issue_pv(i, vs, 1, true);
         return true;
       };
       // with fused RoPE the softmax warpgroups rotate Q in place first
       auto bar_q = [&](int i) { return fused_rope ? bar_q_ready(i) : bar_q_full(i); };
-      bool ok = mma_wait(bar_q(0), 0, abort_flag, limit) &&
-                mma_wait(bar_kv_full(0), 0, abort_flag, limit);
+      bool ok = mma_wait(bar_q(0), 0, abort_flag, limit, eslot) &&
+                mma_wait(bar_kv_full(0), 0, abort_flag, limit, eslot);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
         tc_commit(bar_s_full(0));
-        ok = mma_wait(bar_q(1), 0, abort_flag, limit);
+        ok = mma_wait(bar_q(1), 0, abort_flag, limit, eslot);
       }
       if (ok) {
         tc_fence_after();
@@ -345,10 +293,10 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int vidx = 2 * j + 1, vs = vidx % KV_STAGES;
         const int kidx = 2 * j + 2, ks = kidx % KV_STAGES;
         const bool more = j + 1 < nkv;
-        if (!mma_wait(bar_kv_full(vs), (vidx / KV_STAGES) & 1, abort_flag, limit)) break;
+        if (!mma_wait(bar_kv_full(vs), (vidx / KV_STAGES) & 1, abort_flag, limit, eslot)) break;
         if (!issue_pv_tile(0, vs, j)) break;
         if (more) {
-          if (!mma_wait(bar_kv_full(ks), (kidx / KV_STAGES) & 1, abort_flag, limit)) break;
+          if (!mma_wait(bar_kv_full(ks), (kidx / KV_STAGES) & 1, abort_flag, limit, eslot)) break;
           tc_fence_after();
           issue_s(0, ks);
           tc_commit(bar_s_full(0));
@@ -368,7 +316,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       // Drain: all MMAs issued above complete before TMEM is released.
       tc_commit(bar_mma_done);
       volatile uint32_t never = 0u;
-      mma_wait(bar_mma_done, 0, &never, p.drain_limit_ns);
+      mma_wait(bar_mma_done, 0, &never, p.drain_limit_ns, eslot);
     }
   } else {
     // -------------------------------------------------------- softmax ----
@@ -418,7 +366,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // per row, with the rope kernel's arithmetic (rope_cos_sin, rot2), then
     // make the generic-proxy writes visible to the tensor core (async proxy).
     if (fused_rope) {
-      if (!warp_wait(bar_q_full(wg), 0, abort_flag, limit)) ok = false;
+      if (!warp_wait(bar_q_full(wg), 0, abort_flag, limit, eslot)) ok = false;
       const int row = q_row0 + wg * BM + row_in_tile;
       if (ok && row < p.n_rows) {
         const float* crd = p.coords + (static_cast<long long>(batch) * p.n_rows + row) * 3;
@@ -454,7 +402,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
 
     for (int j = 0; j < nkv; ++j) {
-      if (!warp_wait(bar_s_full(wg), j & 1, abort_flag, limit)) { ok = false; break; }
+      if (!warp_wait(bar_s_full(wg), j & 1, abort_flag, limit, eslot)) { ok = false; break; }
       tc_fence_after();
       const bool last = j == nkv - 1;
       float ls_a;
@@ -502,7 +450,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (__any_sync(0xffffffffu, need)) {
           // the first half of PV(j) may be in flight: let it land, then rescale
           // O (which now includes it) together with the running sum
-          if (!warp_wait(bar_pva_done(wg), j & 1, abort_flag, limit)) { ok = false; break; }
+          if (!warp_wait(bar_pva_done(wg), j & 1, abort_flag, limit, eslot)) { ok = false; break; }
           tc_fence_after();
           float f = 1.f;
           if (need) {
@@ -521,7 +469,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
 
     // epilogue: O / l -> bf16 -> global; optional log-sum-exp
-    if (ok && warp_wait(bar_o_full(wg), 0, abort_flag, limit)) {
+    if (ok && warp_wait(bar_o_full(wg), 0, abort_flag, limit, eslot)) {
       tc_fence_after();
       const int row = q_row0 + wg * BM + row_in_tile;
       const float inv_l = 1.f / l_sum;

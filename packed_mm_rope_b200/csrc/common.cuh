@@ -14,19 +14,26 @@
 
 namespace h3 {
 
-// Device error word bits (one word per device, see h3_check_device_error).
+// Device error word bits (see h3_check_device_error).
 enum : unsigned int {
   DEVERR_TIMEOUT = 1u,
   DEVERR_INPUT = 2u,
 };
 
-__device__ unsigned int g_error_word;
-__device__ unsigned int g_error_snapshot;   // last value taken by take_error_word
+// One error word per stream slot: the host maps each (device, stream) pair it
+// sees to a slot (slot 0 is shared by the streams beyond the table's size) and
+// passes the slot to every kernel it launches on that stream, so a fault is
+// reported by the check of the stream that ran the faulting kernel.
+constexpr int ERR_SLOTS = 256;
+__device__ unsigned int g_error_words[ERR_SLOTS];
+__device__ unsigned int g_error_snapshot[ERR_SLOTS];   // last value taken per slot
 
-// Read and clear the error word in one atomic step, so that a bit raised by a
-// kernel running concurrently on another stream is never lost between the
-// read and the clear.
-__global__ void take_error_word() { g_error_snapshot = atomicExch(&g_error_word, 0u); }
+__device__ __forceinline__ void raise_error(int slot, unsigned int bits) { atomicOr(&g_error_words[slot], bits); }
+
+// Read and clear one slot's word in one atomic step, so that a bit raised by
+// a kernel still running elsewhere is never lost between the read and the
+// clear.
+__global__ void take_error_word(int slot) { g_error_snapshot[slot] = atomicExch(&g_error_words[slot], 0u); }
 
 // ------------------------------------------------------------ timing ----
 
@@ -88,7 +95,7 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 // suspended, so it sees the phase complete within a few cycles.  For waits on
 // the critical path of a single issuing thread.
 __device__ __forceinline__ bool mbar_spin_bounded(uint32_t bar, uint32_t parity,
-                                                  volatile uint32_t* abort, uint64_t limit_ns) {
+                                                  volatile uint32_t* abort, uint64_t limit_ns, int err_slot) {
   if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
@@ -97,7 +104,7 @@ __device__ __forceinline__ bool mbar_spin_bounded(uint32_t bar, uint32_t parity,
     if (*abort) return false;
     if (globaltimer_ns() - t0 > limit_ns) {
       *abort = 1u;
-      atomicOr(&g_error_word, DEVERR_TIMEOUT);
+      raise_error(err_slot, DEVERR_TIMEOUT);
       return false;
     }
   }
@@ -105,9 +112,9 @@ __device__ __forceinline__ bool mbar_spin_bounded(uint32_t bar, uint32_t parity,
 
 // Wait until the phase with `parity` has completed.  Gives up (returns false)
 // when `*abort` becomes non-zero or after `limit_ns` of global time; in the
-// latter case it raises `*abort` and the device error word.
+// latter case it raises `*abort` and the error word of `err_slot`.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                                  volatile uint32_t* abort, uint64_t limit_ns) {
+                                                  volatile uint32_t* abort, uint64_t limit_ns, int err_slot) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
@@ -116,7 +123,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     if (*abort) return false;
     if (globaltimer_ns() - t0 > limit_ns) {
       *abort = 1u;
-      atomicOr(&g_error_word, DEVERR_TIMEOUT);
+      raise_error(err_slot, DEVERR_TIMEOUT);
       return false;
     }
   }

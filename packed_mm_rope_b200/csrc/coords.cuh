@@ -42,7 +42,7 @@ __device__ __forceinline__ float canvas(long long idx, int n, int gh, int gw) {
 }
 
 __global__ void __launch_bounds__(256) coords_kernel(const CoordTable tab, const int32_t* perm,
-                                                     long long n_rows, float* out) {
+                                                     long long n_rows, float* out, int err_slot) {
   const long long step = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long r = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; r < n_rows;
        r += step) {
@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(256) coords_kernel(const CoordTable tab, const
     if (perm != nullptr) {
       e = perm[r];
       if (e < 0 || e >= n_rows) {
-        atomicOr(&g_error_word, DEVERR_INPUT);
+        raise_error(err_slot, DEVERR_INPUT);
         const float nan = __int_as_float(0x7fc00000);
         out[3 * r + 0] = nan;
         out[3 * r + 1] = nan;

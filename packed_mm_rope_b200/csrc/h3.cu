@@ -26,21 +26,22 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
-// One-time set-up of the current device, kept for the life of the process:
-// the shared-memory opt-ins of the kernels that need more than 48 KB
-// (function attributes are per device) and the SM count.
+// One-time set-up of the current device, kept until h3_shutdown: the
+// shared-memory opt-ins of the kernels that need more than 48 KB (function
+// attributes are per device) and the SM count.
 struct DeviceState {
   bool ready = false;
   int sms = 148;
 };
 
+std::mutex g_state_mu;
+DeviceState g_states[64];
+
 const DeviceState* device_state() {
-  static std::mutex mu;
-  static DeviceState states[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  DeviceState& st = states[dev];
+  std::lock_guard<std::mutex> lock(g_state_mu);
+  DeviceState& st = g_states[dev];
   if (!st.ready) {
     if (cudaFuncSetAttribute(h3::attn::attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(h3::attn::SMEM_BYTES)) != cudaSuccess)
@@ -55,6 +56,26 @@ const DeviceState* device_state() {
 int sm_count() {
   const DeviceState* st = device_state();
   return st ? st->sms : 148;
+}
+
+// Error-word slot of (current device, stream).  Slots 1 .. ERR_SLOTS-1 are
+// handed out to streams in the order they are first seen; once they are used
+// up, further streams share slot 0.  A stream destroyed and re-created at the
+// same address keeps its slot.  Forgotten by h3_shutdown.
+std::mutex g_slot_mu;
+void* g_slot_stream[64][h3::ERR_SLOTS];
+int g_slots_used[64];
+
+int error_slot(void* stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(g_slot_mu);
+  for (int i = 1; i <= g_slots_used[dev]; ++i)
+    if (g_slot_stream[dev][i] == stream) return i;
+  if (g_slots_used[dev] + 1 >= h3::ERR_SLOTS) return 0;
+  const int i = ++g_slots_used[dev];
+  g_slot_stream[dev][i] = stream;
+  return i;
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -118,37 +139,14 @@ h3::RopeTable make_rope_table(const h3_rope_cfg* cfg) {
   return t;
 }
 
-}  // namespace
-
-extern "C" {
-
-const char* h3_status_str(int32_t status) {
-  switch (status) {
-    case H3_OK: return "ok";
-    case H3_ERR_INVALID_ARG: return "invalid argument";
-    case H3_ERR_UNSUPPORTED: return "unsupported argument";
-    case H3_ERR_CUDA: return "CUDA error";
-    case H3_ERR_TIMEOUT: return "bounded device wait expired";
-    case H3_ERR_DEVICE_INPUT: return "kernel found an invalid input";
-    case H3_ERR_TOO_LARGE: return "problem exceeds the fixed scratch of the no-allocation call";
-    default: return "unknown status";
-  }
-}
-
-int32_t h3_version(void) { return 101; }
-
-h3_status h3_set_wait_limit_ns(uint64_t ns) {
-  g_wait_limit_ns.store(ns == 0 ? kDefaultWaitLimitNs : ns);
-  return H3_OK;
-}
-
-h3_status h3_build_coords(const h3_segment* segs, int32_t nseg, const int32_t* d_perm, int64_t n_rows,
-                          float* d_coords, void* stream) {
+// Checks a segment table against n_rows and packs it for the coordinate
+// kernel; nothing is launched.  Every host-buffer call runs this before it
+// queues any work, so a bad table never leaves copies in flight.
+h3_status make_coord_table(const h3_segment* segs, int32_t nseg, int64_t n_rows, h3::CoordTable* tab) {
   if (segs == nullptr || nseg < 1 || nseg > H3_MAX_SEGMENTS || n_rows < 0) return H3_ERR_INVALID_ARG;
   static_assert(sizeof(h3::CoordTable) <= 4000, "segment table must fit in kernel parameters");
-  h3::CoordTable tab;
-  std::memset(&tab, 0, sizeof(tab));
-  tab.nseg = nseg;
+  std::memset(tab, 0, sizeof(*tab));
+  tab->nseg = nseg;
   long long first = 0;
   constexpr long long kExact = 1ll << 24;   // integers below this are exact in fp32
   for (int i = 0; i < nseg; ++i) {
@@ -175,19 +173,51 @@ h3_status h3_build_coords(const h3_segment* segs, int32_t nseg, const int32_t* d
       const long long t1 = s.t_off_num + static_cast<long long>(s.count - 1) * s.t_step_num;
       if (t0 <= -kExact || t0 >= kExact || t1 <= -kExact || t1 >= kExact) return H3_ERR_INVALID_ARG;
     }
-    tab.seg[i] = s;
-    tab.first[i] = first;
+    tab->seg[i] = s;
+    tab->first[i] = first;
     first += rows;
     if (first > (1ll << 40)) return H3_ERR_INVALID_ARG;
   }
-  tab.first[nseg] = first;
-  if (first != n_rows) return H3_ERR_INVALID_ARG;
+  tab->first[nseg] = first;
+  return first == n_rows ? H3_OK : H3_ERR_INVALID_ARG;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* h3_status_str(int32_t status) {
+  switch (status) {
+    case H3_OK: return "ok";
+    case H3_ERR_INVALID_ARG: return "invalid argument";
+    case H3_ERR_UNSUPPORTED: return "unsupported argument";
+    case H3_ERR_CUDA: return "CUDA error";
+    case H3_ERR_TIMEOUT: return "bounded device wait expired";
+    case H3_ERR_DEVICE_INPUT: return "kernel found an invalid input";
+    case H3_ERR_TOO_LARGE: return "problem exceeds the fixed scratch of the no-allocation call";
+    default: return "unknown status";
+  }
+}
+
+int32_t h3_version(void) { return 101; }
+
+h3_status h3_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns.store(ns == 0 ? kDefaultWaitLimitNs : ns);
+  return H3_OK;
+}
+
+h3_status h3_build_coords(const h3_segment* segs, int32_t nseg, const int32_t* d_perm, int64_t n_rows,
+                          float* d_coords, void* stream) {
+  h3::CoordTable tab;
+  const h3_status st = make_coord_table(segs, nseg, n_rows, &tab);
+  if (st != H3_OK) return st;
   if (n_rows == 0) return H3_OK;
   if (d_coords == nullptr) return H3_ERR_INVALID_ARG;
   const int threads = 256;
   const long long blocks_needed = (n_rows + threads - 1) / threads;
   const int blocks = static_cast<int>(blocks_needed < 8LL * sm_count() ? blocks_needed : 8LL * sm_count());
-  h3::coords_kernel<<<blocks, threads, 0, as_stream(stream)>>>(tab, d_perm, n_rows, d_coords);
+  h3::coords_kernel<<<blocks, threads, 0, as_stream(stream)>>>(tab, d_perm, n_rows, d_coords,
+                                                               error_slot(stream));
   return cudaGetLastError() == cudaSuccess ? H3_OK : H3_ERR_CUDA;
 }
 
@@ -260,6 +290,7 @@ h3_status h3_packed_attention(const void* d_q, const void* d_k, const void* d_v,
   p.lse = d_lse;
   p.wait_limit_ns = g_wait_limit_ns.load();
   p.drain_limit_ns = kDrainLimitNs;
+  p.err_slot = error_slot(stream);
   p.coords = d_coords;
   p.rope_layout = d_coords ? cfg->pair_layout : 0;
   if (d_coords) p.rope = make_rope_table(cfg);
@@ -287,7 +318,7 @@ h3_status h3_adaln_modulate(const void* d_x, void* d_y, const int32_t* d_timeste
   h3::adaln_kernel<<<static_cast<int>(grid), h3::ADALN_THREADS, 0, as_stream(stream)>>>(
       static_cast<const uint4*>(d_x), static_cast<uint4*>(d_y), d_timestep_index, d_token_tag,
       reinterpret_cast<const float4*>(d_table), n_entries, n_rows, hidden / 8, x_row_stride / 8, y_row_stride / 8,
-      eps);
+      eps, error_slot(stream));
   return cudaGetLastError() == cudaSuccess ? H3_OK : H3_ERR_CUDA;
 }
 
@@ -378,12 +409,19 @@ h3_status h3_packed_mmrope_attention_host(const h3_segment* segs, int32_t nseg, 
                                           const void* h_q, const void* h_k, const void* h_v, void* h_o,
                                           void* d_work, int64_t n_rows, int32_t n_heads,
                                           int32_t heads_per_chunk, const h3_rope_cfg* cfg, void* stream) {
+  // every argument is checked before anything is queued
   if (n_rows < 0 || n_heads < 1 || !valid_rope_cfg(cfg)) return H3_ERR_INVALID_ARG;
   if (cfg->head_dim != 128) return H3_ERR_UNSUPPORTED;
   if (heads_per_chunk < 0 || heads_per_chunk > n_heads) return H3_ERR_INVALID_ARG;
-  if (n_rows == 0) return h3_build_coords(segs, nseg, nullptr, 0, nullptr, stream);
+  h3::CoordTable tab;
+  h3_status st = make_coord_table(segs, nseg, n_rows, &tab);
+  if (st != H3_OK || n_rows == 0) return st;
   if (!h_q || !h_k || !h_v || !h_o) return H3_ERR_INVALID_ARG;
+  if (n_rows >= (1ll << 31)) return H3_ERR_INVALID_ARG;
   if (d_work == nullptr || (reinterpret_cast<uintptr_t>(d_work) & 255u)) return H3_ERR_INVALID_ARG;
+  const int hc = heads_per_chunk > 0 ? heads_per_chunk : pick_heads_per_chunk(n_rows, n_heads);
+  const int nchunks = (n_heads + hc - 1) / hc;
+  if (nchunks > 64) return H3_ERR_UNSUPPORTED;
   HostPipe* hp = host_pipe();
   if (hp == nullptr) return H3_ERR_CUDA;
   std::lock_guard<std::mutex> lock(hp->enqueue);
@@ -398,13 +436,18 @@ h3_status h3_packed_mmrope_attention_host(const h3_segment* segs, int32_t nseg, 
   float* dcoords = reinterpret_cast<float*>(w + 4 * t);
   int32_t* dperm = reinterpret_cast<int32_t*>(w + 4 * t + up(static_cast<uint64_t>(n_rows) * 12u));
 
-  const int hc = heads_per_chunk > 0 ? heads_per_chunk : pick_heads_per_chunk(n_rows, n_heads);
-  const int nchunks = (n_heads + hc - 1) / hc;
-  if (nchunks > 64) return H3_ERR_UNSUPPORTED;
   cudaEvent_t* ev_in = hp->ev;
   cudaEvent_t* ev_out = hp->ev + 64;
   cudaEvent_t ev_start = hp->ev[192], ev_end = hp->ev[193];
   auto ck = [](cudaError_t e) { return e == cudaSuccess; };
+  // After a failure with copies already queued: order `stream` after both copy
+  // streams, so that a caller who synchronises `stream` and then frees its
+  // host buffers cannot race a copy still in flight.
+  auto fail = [&](h3_status status) {
+    if (ck(cudaEventRecord(ev_end, hp->h2d))) cudaStreamWaitEvent(s, ev_end, 0);
+    if (ck(cudaEventRecord(ev_start, hp->d2h))) cudaStreamWaitEvent(s, ev_start, 0);
+    return status;
+  };
 
   // both copy streams start after the work already queued on `stream`
   if (!ck(cudaEventRecord(ev_start, s)) || !ck(cudaStreamWaitEvent(hp->h2d, ev_start, 0)) ||
@@ -413,10 +456,10 @@ h3_status h3_packed_mmrope_attention_host(const h3_segment* segs, int32_t nseg, 
   // coordinates (after the permutation is on the device)
   if (h_perm != nullptr) {
     if (!ck(cudaMemcpyAsync(dperm, h_perm, static_cast<size_t>(n_rows) * 4, cudaMemcpyHostToDevice, s)))
-      return H3_ERR_CUDA;
+      return fail(H3_ERR_CUDA);
   }
-  h3_status st = h3_build_coords(segs, nseg, h_perm ? dperm : nullptr, n_rows, dcoords, stream);
-  if (st != H3_OK) return st;
+  st = h3_build_coords(segs, nseg, h_perm ? dperm : nullptr, n_rows, dcoords, stream);
+  if (st != H3_OK) return fail(st);
 
   for (int c = 0; c < nchunks; ++c) {
     const int h0 = c * hc, nh = (h0 + hc <= n_heads) ? hc : n_heads - h0;
@@ -426,23 +469,25 @@ h3_status h3_packed_mmrope_attention_host(const h3_segment* segs, int32_t nseg, 
       uint8_t* dst = (x == 0 ? dq : x == 1 ? dk : dv) + off;
       if (!ck(cudaMemcpy2DAsync(dst, row_bytes, src, row_bytes, width, static_cast<size_t>(n_rows),
                                 cudaMemcpyHostToDevice, hp->h2d)))
-        return H3_ERR_CUDA;
+        return fail(H3_ERR_CUDA);
     }
-    if (!ck(cudaEventRecord(ev_in[c], hp->h2d)) || !ck(cudaStreamWaitEvent(s, ev_in[c], 0))) return H3_ERR_CUDA;
+    if (!ck(cudaEventRecord(ev_in[c], hp->h2d)) || !ck(cudaStreamWaitEvent(s, ev_in[c], 0)))
+      return fail(H3_ERR_CUDA);
     // rotate this chunk's Q and K in place, then attend over all rows for its heads
     st = h3_mmrope_qk(dq + off, dk + off, dq + off, dk + off, dcoords, n_rows, nh,
                       static_cast<int64_t>(n_heads) * 128, cfg, stream);
-    if (st != H3_OK) return st;
+    if (st != H3_OK) return fail(st);
     st = h3_packed_attention(dq + off, dk + off, dv + off, d_o + off, nullptr, nullptr, nullptr, 1, n_rows, nh, 128,
                              static_cast<int64_t>(n_heads) * 128, 0.f, stream);
-    if (st != H3_OK) return st;
-    if (!ck(cudaEventRecord(ev_out[c], s)) || !ck(cudaStreamWaitEvent(hp->d2h, ev_out[c], 0))) return H3_ERR_CUDA;
+    if (st != H3_OK) return fail(st);
+    if (!ck(cudaEventRecord(ev_out[c], s)) || !ck(cudaStreamWaitEvent(hp->d2h, ev_out[c], 0)))
+      return fail(H3_ERR_CUDA);
     if (!ck(cudaMemcpy2DAsync(static_cast<uint8_t*>(h_o) + off, row_bytes, d_o + off, row_bytes, width,
                               static_cast<size_t>(n_rows), cudaMemcpyDeviceToHost, hp->d2h)))
-      return H3_ERR_CUDA;
+      return fail(H3_ERR_CUDA);
   }
   // `stream` is ordered after the last copy out (and, through it, all others)
-  if (!ck(cudaEventRecord(ev_end, hp->d2h)) || !ck(cudaStreamWaitEvent(s, ev_end, 0))) return H3_ERR_CUDA;
+  if (!ck(cudaEventRecord(ev_end, hp->d2h)) || !ck(cudaStreamWaitEvent(s, ev_end, 0))) return fail(H3_ERR_CUDA);
   return H3_OK;
 }
 
@@ -458,20 +503,22 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[H3_NOALLOC_SCRA
 
 namespace {
 
-// Device address of g_noalloc_scratch on the current device (cached per
-// device after the first lookup), or null if the lookup fails.
+std::mutex g_scratch_mu;
+void* g_scratch_addr[64];
+
+// Device address of g_noalloc_scratch on the current device (looked up on the
+// first call per device and cached until h3_shutdown), or null if the lookup
+// fails.  A device reset moves the array, hence h3_shutdown before any reset.
 void* noalloc_scratch() {
-  static std::mutex mu;
-  static void* addr[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = p;
+    g_scratch_addr[dev] = p;
   }
-  return addr[dev];
+  return g_scratch_addr[dev];
 }
 
 }  // namespace
@@ -482,9 +529,12 @@ h3_status h3_packed_mmrope_attention_host_noalloc(const h3_segment* segs, int32_
                                                   const void* h_q, const void* h_k, const void* h_v, void* h_o,
                                                   int64_t n_rows, int32_t n_heads, const h3_rope_cfg* cfg,
                                                   void* stream) {
+  // every argument is checked before anything is queued
   if (n_rows < 0 || n_heads < 1 || !valid_rope_cfg(cfg)) return H3_ERR_INVALID_ARG;
   if (cfg->head_dim != 128) return H3_ERR_UNSUPPORTED;
-  if (n_rows == 0) return h3_build_coords(segs, nseg, nullptr, 0, nullptr, stream);
+  h3::CoordTable tab;
+  const h3_status tst = make_coord_table(segs, nseg, n_rows, &tab);
+  if (tst != H3_OK || n_rows == 0) return tst;
   if (!h_q || !h_k || !h_v || !h_o) return H3_ERR_INVALID_ARG;
   const uint64_t need = h3_host_workspace_bytes(n_rows, n_heads);
   if (need == 0) return H3_ERR_INVALID_ARG;
@@ -521,12 +571,14 @@ h3_status h3_packed_mmrope_attention_host_noalloc(const h3_segment* segs, int32_
 }
 
 h3_status h3_check_device_error(void* stream) {
-  // ordered after the work already on `stream`
-  h3::take_error_word<<<1, 1, 0, as_stream(stream)>>>();
+  // this stream's word, taken by a kernel ordered after the work already on it
+  const int slot = error_slot(stream);
+  h3::take_error_word<<<1, 1, 0, as_stream(stream)>>>(slot);
   if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(as_stream(stream)) != cudaSuccess)
     return H3_ERR_CUDA;
   unsigned int word = 0;
-  if (cudaMemcpyFromSymbol(&word, h3::g_error_snapshot, sizeof(word)) != cudaSuccess) return H3_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&word, h3::g_error_snapshot, sizeof(word), sizeof(word) * slot) != cudaSuccess)
+    return H3_ERR_CUDA;
   if (word & h3::DEVERR_TIMEOUT) return H3_ERR_TIMEOUT;
   if (word & h3::DEVERR_INPUT) return H3_ERR_DEVICE_INPUT;
   return H3_OK;
@@ -565,14 +617,28 @@ h3_status h3_init(int32_t device) {
   if (encode_tiled() == nullptr || device_state() == nullptr || host_pipe() == nullptr ||
       noalloc_scratch() == nullptr)
     return H3_ERR_CUDA;
-  const unsigned int zero = 0;
-  if (cudaMemcpyToSymbol(h3::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return H3_ERR_CUDA;
+  static const unsigned int zeros[h3::ERR_SLOTS] = {};
+  if (cudaMemcpyToSymbol(h3::g_error_words, zeros, sizeof(zeros)) != cudaSuccess) return H3_ERR_CUDA;
   return H3_OK;
 }
 
 void h3_shutdown(void) {
   DeviceGuard guard;
   release_host_pipes();
+  // per-device lookups and set-up are redone by the next call (after a device
+  // reset the module, its kernels' attributes and its arrays are new)
+  {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    for (auto& a : g_scratch_addr) a = nullptr;
+  }
+  {
+    std::lock_guard<std::mutex> lock(g_state_mu);
+    for (auto& st : g_states) st = DeviceState();
+  }
+  {
+    std::lock_guard<std::mutex> lock(g_slot_mu);
+    for (auto& n : g_slots_used) n = 0;
+  }
 }
 
 }  // extern "C"

@@ -122,3 +122,19 @@ def test_init_without_a_device_fails_cleanly():
     assert _err(h3.h3_init, 0) in (h3.H3_ERR_CUDA, h3.H3_ERR_INVALID_ARG)
     h3.h3_shutdown()
     assert _lib.load().h3_version() == 101
+
+
+def test_host_calls_check_the_segment_table_before_queuing_anything():
+    # A table that does not add up to n_rows is refused before any copy is
+    # queued: the host pointers (never dereferenced) and the missing GPU are
+    # not reached, so the status is INVALID_ARG, not a CUDA error.
+    P, WORK = 0x10000, 0x100000
+    cfg = h3.rope_cfg()
+    for segs, n in (([W.text(4)], 5), ([W.Segment(W.SEG_TEXT, 4, t_den=0)], 4), ([W.text(1)] * 65, 65)):
+        assert _err(h3.h3_packed_mmrope_attention_host, segs, 0, P, P, P, P, WORK, n, 1, cfg) == \
+            h3.H3_ERR_INVALID_ARG
+        assert _err(_lib.h3_packed_mmrope_attention_host_noalloc, segs, 0, P, P, P, P, n, 1, cfg) == \
+            h3.H3_ERR_INVALID_ARG
+    # too many head chunks is also refused up front
+    assert _err(h3.h3_packed_mmrope_attention_host, [W.text(4)], 0, P, P, P, P, WORK, 4, 65, cfg, 1) == \
+        h3.H3_ERR_UNSUPPORTED

@@ -5,8 +5,9 @@ slack); attention within max |err| <= 2e-2, mean |err| <= 2e-3 and relative
 error <= 1e-2 against the oracle on the same bf16 inputs.  Small workloads
 are compared in full; the three large ones (28,196 / 81,792 / 31,952 rows x
 42 heads) run in full on the GPU in the benchmark's launch configuration and
-are compared on seeded sampled query rows (every segment kind, rows 0 and
-N-1, the whole last partial tile) for four heads.
+are compared on >= 2,048 seeded query rows (every segment kind, rows 0 and
+N-1, the whole last partial tile, a row in every 256-row block) for all 42
+heads.
 """
 import numpy as np
 import pytest
@@ -122,9 +123,15 @@ def test_rope_single_frequency_ladder(h3, layout):
         assert frac_rne > 0.99
 
 
-def test_rope_parity_worked_example_sampled(h3):
-    wl = W.workload(2)
-    for frac_rne, _ in _rope_case(h3, wl, rows=W.sample_rows(wl, 200)):
+@pytest.mark.slow
+@pytest.mark.parametrize("cfg", [2, 3, 4])
+def test_rope_parity_full_size_sampled(h3, cfg):
+    # the three large workloads, rotated in full on the GPU; compared on 2,048
+    # seeded rows x all heads (plus every segment's first, middle and last row
+    # and the last partial tile).  Workload 4 holds the largest |t| (reference
+    # audio at -2000 (c + 1) + j, down to about -6,000): the angle-precision case.
+    wl = W.workload(cfg)
+    for frac_rne, _ in _rope_case(h3, wl, rows=W.sample_rows(wl, 2048)):
         assert frac_rne > 0.99
 
 
@@ -218,17 +225,29 @@ def test_pipeline_peaky_queries(h3):
     check_attention(got, ref, "peaky x4", logit_scale=4.0)
 
 
+def _rows_covering_every_block(wl, n, block=256):
+    """W.sample_rows(wl, n) plus one seeded row in every ``block``-row range, so
+    that every (query block, head) CTA of the attention grid has a checked row."""
+    N = wl.n_rows
+    nb = (N + block - 1) // block
+    off = (W.uniform01(wl.seed, 11, nb) * block).astype(np.int64)
+    per_block = np.minimum(np.arange(nb, dtype=np.int64) * block + off, N - 1)
+    return np.union1d(W.sample_rows(wl, n), per_block)
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("cfg", [2, 3, 4])
 def test_pipeline_parity_full_size_sampled(h3, cfg):
+    # the whole path in full on the GPU, in the launch configuration the
+    # benchmark times; compared element by element with the fp64 oracle on
+    # >= 2,048 seeded query rows x ALL heads (every CTA of the grid covered)
     wl = W.workload(cfg)
     q, k, v = W.qkv_bf16(wl)
     perm, got = _pipeline(h3, wl, q, k, v)
-    rows = W.sample_rows(wl, 96)
-    heads = sorted({0, 1, wl.heads // 2, wl.heads - 1})
-    ref, _ = opipe.packed_mmrope_attention(wl.segments, perm, q, k, v, wl.theta, wl.sections,
-                                           rows=rows, heads=heads)
-    check_attention(got[rows][:, heads], ref, wl.name)
+    rows = _rows_covering_every_block(wl, 2048)
+    assert rows.size >= 2048
+    ref, _ = opipe.packed_mmrope_attention(wl.segments, perm, q, k, v, wl.theta, wl.sections, rows=rows)
+    check_attention(got[rows], ref, wl.name)
 
 
 def test_row_order_carries_no_position_on_gpu(h3):

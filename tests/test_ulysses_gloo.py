@@ -50,7 +50,7 @@ def _worker(rank, world, port, heads, out):
     dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,heads", [(2, 5), (3, 5), (3, 2)])
+@pytest.mark.parametrize("world,heads", [(2, 5), (3, 5), (3, 2), (4, 42)])
 def test_ulysses_matches_whole_sequence(world, heads):
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
@@ -67,7 +67,7 @@ def test_ulysses_matches_whole_sequence(world, heads):
 
 def test_even_split():
     from packed_mm_rope_b200.ulysses import even_split
-    assert even_split(42, 4) == [11, 11, 10, 10]
+    assert even_split(42, 4) == [11, 11, 10, 10]      # the pages' 4-GPU deployment of 42 heads
     assert even_split(82, 3) == [28, 27, 27]
     assert even_split(2, 3) == [1, 1, 0]
     with pytest.raises(ValueError):
