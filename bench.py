@@ -153,6 +153,7 @@ def run_ours(args):
     dq, dk, dv = (t.to(dev) for t in (hq, hk, hv))
     dqr, dkr, do = torch.empty_like(dq), torch.empty_like(dk), torch.empty_like(dq)
     coords = torch.empty((N, 3), dtype=torch.float32, device=dev)
+    rope_cs = torch.empty((N, 64, 2), dtype=torch.float32, device=dev) if args.fused_q_rope else None
     hperm = None if perm is None else torch.from_numpy(perm.astype(np.int32)).pin_memory()
     dperm = None if perm is None else hperm.to(dev)
     stream = torch.cuda.current_stream(dev)
@@ -176,7 +177,9 @@ def run_ours(args):
         if evs is not None:
             evs[1].record(stream)
         if fused:
-            # K rotated by the rope kernel, Q rotated inside the attention kernel
+            # the rows' rotary table, K rotated by the rope kernel, Q rotated
+            # inside the attention kernel from the table
+            call(L.h3_rope_cos_sin(coords.data_ptr(), N, cfg, rope_cs.data_ptr(), s), "h3_rope_cos_sin")
             call(L.h3_mmrope_qk(None, dk.data_ptr(), None, dkr.data_ptr(), coords.data_ptr(),
                                 N, H, rs, cfg, s), "h3_mmrope_qk")
         else:
@@ -186,7 +189,7 @@ def run_ours(args):
             evs[2].record(stream)
         if fused:
             call(L.h3_packed_attention(dq.data_ptr(), dkr.data_ptr(), dv.data_ptr(), do.data_ptr(), None,
-                                       coords.data_ptr(), cfg, 1, N, H, D, rs, 0.0, s), "h3_packed_attention")
+                                       rope_cs.data_ptr(), cfg, 1, N, H, D, rs, 0.0, s), "h3_packed_attention")
         else:
             call(L.h3_packed_attention(dqr.data_ptr(), dkr.data_ptr(), dv.data_ptr(), do.data_ptr(), None, None,
                                        None, 1, N, H, D, rs, 0.0, s), "h3_packed_attention")
@@ -260,7 +263,8 @@ def run_ours(args):
     pk, src = peaks()
     value = hdist.weak_scaling_throughput(flops, world, ms_per_step * 1e-3) / 1e12
     attn_tflops = flops / (attn_ms_max * 1e-3) / 1e12
-    rope_bytes = (2 if fused else 4) * N * H * D * 2 + N * 12
+    # fused: K read + written, coords read twice, the (cos, sin) table written
+    rope_bytes = (2 * N * H * D * 2 + N * 24 + N * 512) if fused else (4 * N * H * D * 2 + N * 12)
     rope_gbs = rope_bytes / (rope_ms * 1e-3) / 1e9
     traffic = profiled_traffic(wl)
     line = {
@@ -284,12 +288,13 @@ def run_ours(args):
                      "traffic": traffic},
         "rope": {"kernel": "h3_mmrope_qk", "bound": "hbm", "achieved": round(rope_gbs, 1), "peak": pk["hbm_gbs"],
                  "unit": "GB/s", "frac": round(rope_gbs / pk["hbm_gbs"], 4),
-                 "algorithmic": "4*N*H*D*2 + 12*N = %d bytes per launch" % rope_bytes},
+                 "algorithmic": ("2*N*H*D*2 + 24*N + 512*N = %d bytes per step (table + K-only rope)" if fused
+                                 else "4*N*H*D*2 + 12*N = %d bytes per launch") % rope_bytes},
         "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "h3_packed_mmrope_attention_host (pinned host Q/K/V -> host O, copies overlapped with "
                        "compute over chunks of heads)"},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": (4 if fused else 3) * args.steps,
         "clocks": clk.summary(),
     }
     if args.adaln:
@@ -414,7 +419,7 @@ def main():
     ap.add_argument("--video-frames", type=int, default=0,
                     help="resize the worked-example layout to this many latent frames (profiling cases)")
     ap.add_argument("--fused-q-rope", action="store_true",
-                    help="rotate only K in h3_mmrope_qk and Q inside h3_packed_attention")
+                    help="rotate only K in h3_mmrope_qk and Q inside h3_packed_attention (from h3_rope_cos_sin)")
     ap.add_argument("--adaln", action="store_true", help="also time h3_adaln_modulate on [N, H*128]")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=128, help="query rows of the timed oracle sample")

@@ -216,6 +216,24 @@ h3_status h3_mmrope_qk(const void* d_q, const void* d_k, void* d_q_out, void* d_
                        int64_t row_stride, const h3_rope_cfg* cfg, void* stream);
 
 /*
+ * h3_rope_cos_sin -- the rotary table of every row: for pair p of row r,
+ * d_cs[r][p] = (cos a, sin a), a = fp64(coordinate of p's axis) x fp64
+ * inverse frequency of p, fp64 sincos, each rounded to fp32: exactly the
+ * values h3_mmrope_qk rotates by.  Defining passages: as h3_mmrope_qk.  It is
+ * the input of h3_packed_attention's fused Q rotation, which then rotates
+ * with a table read instead of recomputing the trigonometry in every CTA.
+ *
+ *   d_coords   device float[n_rows][3] from h3_build_coords
+ *   n_rows     rows (batch folded in)
+ *   cfg        host rotary configuration (head_dim 128: 64 pairs per row)
+ *   d_cs       device float[n_rows][64][2], 16-byte aligned, written
+ * Errors: H3_ERR_INVALID_ARG (NULL pointer with n_rows > 0, bad cfg);
+ * H3_ERR_UNSUPPORTED (head_dim != 128, misaligned d_cs).
+ */
+h3_status h3_rope_cos_sin(const float* d_coords, int64_t n_rows, const h3_rope_cfg* cfg, float* d_cs,
+                          void* stream);
+
+/*
  * h3_packed_attention -- full (non-causal, unmasked) softmax attention over
  * all packed rows, per batch and head:  O = softmax(Q K^T * scale) V.
  * Defining passages: [P1] sections 2 and 6 (one packed sequence, full
@@ -226,10 +244,11 @@ h3_status h3_mmrope_qk(const void* d_q, const void* d_k, void* d_q_out, void* d_
  *   d_o             device bf16 output, same layout and row_stride
  *   d_lse           device float[batch][n_heads][n_rows] natural-log row
  *                   log-sum-exp of the scaled logits, or NULL
- *   d_coords, cfg   NULL: Q and K arrive rotated.  Non-NULL (device float
- *                   [batch][n_rows][3] from h3_build_coords, host cfg): Q arrives
- *                   UNROTATED and each CTA rotates its Q tiles in shared memory
- *                   as they are loaded, with exactly the arithmetic of
+ *   d_rope_cs, cfg  NULL: Q and K arrive rotated.  Non-NULL (device float
+ *                   [batch][n_rows][64][2] from h3_rope_cos_sin, 16-byte aligned;
+ *                   host cfg for its pair layout): Q arrives UNROTATED and each
+ *                   CTA rotates its Q tiles in shared memory as they are loaded,
+ *                   with the table's (cos, sin) and exactly the arithmetic of
  *                   h3_mmrope_qk (so O is identical to rotating first); K must
  *                   already be rotated (h3_mmrope_qk with d_q = NULL).  Rotating K
  *                   here would repeat the work in every query-tile CTA of a head.
@@ -239,11 +258,11 @@ h3_status h3_mmrope_qk(const void* d_q, const void* d_k, void* d_q_out, void* d_
  * bf16.  All waits inside the kernel are bounded; on expiry the kernel stops
  * and h3_check_device_error returns H3_ERR_TIMEOUT.
  * Errors: H3_ERR_INVALID_ARG (NULL pointers with n_rows > 0, n_rows >= 2^31,
- * batch or n_heads < 1, bad stride, bad cfg with d_coords); H3_ERR_UNSUPPORTED
+ * batch or n_heads < 1, bad stride, bad cfg with d_rope_cs); H3_ERR_UNSUPPORTED
  * (head_dim != 128, misaligned pointer or stride).
  */
 h3_status h3_packed_attention(const void* d_q, const void* d_k, const void* d_v, void* d_o,
-                              float* d_lse, const float* d_coords, const h3_rope_cfg* cfg,
+                              float* d_lse, const float* d_rope_cs, const h3_rope_cfg* cfg,
                               int32_t batch, int64_t n_rows, int32_t n_heads, int32_t head_dim,
                               int64_t row_stride, float softmax_scale, void* stream);
 

@@ -6,6 +6,7 @@ step of the path runs in the library's CUDA kernels:
 
 * ``h3_build_coords``     packed segment table -> per-row (t, h, w) fp32
 * ``h3_mmrope_qk``        three-axis rotary rotation of bf16 Q and K
+* ``h3_rope_cos_sin``     the per-row rotary (cos, sin) table of the fused Q rotation
 * ``h3_packed_attention`` full softmax attention over the packed rows
 
 The library is loaded on first use (``load()``, or any call below) and a
@@ -20,6 +21,7 @@ from ._lib import (H3Error, H3_OK, H3_ERR_INVALID_ARG, H3_ERR_UNSUPPORTED, H3_ER
                    H3_ERR_TIMEOUT, H3_ERR_DEVICE_INPUT, H3_ERR_TOO_LARGE, h3_adaln_modulate,
                    h3_build_coords, h3_check_device_error, h3_init, h3_shutdown,
                    h3_host_workspace_bytes, h3_mmrope_qk, h3_packed_attention, h3_packed_mmrope_attention_host,
+                   h3_rope_cos_sin,
                    h3_set_wait_limit_ns, rope_cfg, status_str)
 
 load = _lib.load
@@ -85,12 +87,29 @@ def mmrope_qk(q, k, coords, q_out=None, k_out=None, theta=10000.0, sections=(32,
     return (q_out if q is not None else None), k_out
 
 
-def packed_attention(q, k, v, out=None, lse=None, softmax_scale: float = 0.0, stream=None, coords=None,
+def rope_cos_sin(coords, out=None, theta=10000.0, sections=(32, 48, 48), pair_layout=0, freq_rule=0,
+                 stream=None):
+    """fp32 [rows, 64, 2] rotary (cos, sin) table of fp32 [rows, 3] coordinates."""
+    import torch
+    if coords.dtype != torch.float32 or coords.dim() != 2 or coords.shape[1] != 3 or not coords.is_contiguous():
+        raise ValueError("coords must be contiguous fp32 [rows, 3]")
+    n = coords.shape[0]
+    if out is None:
+        out = torch.empty((n, 64, 2), dtype=torch.float32, device=coords.device)
+    if out.dtype != torch.float32 or out.numel() != n * 128 or not out.is_contiguous():
+        raise ValueError("out must be contiguous fp32 [rows, 64, 2]")
+    h3_rope_cos_sin(coords.data_ptr(), n, rope_cfg(theta, 128, sections, pair_layout, freq_rule), out.data_ptr(),
+                    _stream(stream))
+    return out
+
+
+def packed_attention(q, k, v, out=None, lse=None, softmax_scale: float = 0.0, stream=None, rope_cs=None,
                      theta=10000.0, sections=(32, 48, 48), pair_layout=0, freq_rule=0):
     """O = softmax(Q K^T * scale) V over all packed rows, per head.
 
-    With ``coords`` (fp32 [rows, 3]) Q is passed UNROTATED and rotated inside
-    the kernel as its tiles are loaded; K must already be rotated.
+    With ``rope_cs`` (fp32 [rows, 64, 2] from ``rope_cos_sin``) Q is passed
+    UNROTATED and rotated inside the kernel as its tiles are loaded; K must
+    already be rotated.
     """
     import torch
     lay = _row_layout(q)
@@ -106,12 +125,12 @@ def packed_attention(q, k, v, out=None, lse=None, softmax_scale: float = 0.0, st
             raise ValueError("lse must be contiguous fp32 [B, H, N]")
         lp = lse.data_ptr()
     cp, cfg = 0, None
-    if coords is not None:
-        if coords.dtype != torch.float32 or coords.numel() != 3 * b * n or not coords.is_contiguous():
-            raise ValueError("coords must be contiguous fp32 [rows, 3]")
-        cp, cfg = coords.data_ptr(), rope_cfg(theta, 128, sections, pair_layout, freq_rule)
+    if rope_cs is not None:
+        if rope_cs.dtype != torch.float32 or rope_cs.numel() != 128 * b * n or not rope_cs.is_contiguous():
+            raise ValueError("rope_cs must be contiguous fp32 [rows, 64, 2]")
+        cp, cfg = rope_cs.data_ptr(), rope_cfg(theta, 128, sections, pair_layout, freq_rule)
     h3_packed_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lp, b, n, h, rs,
-                        softmax_scale, d_coords=cp, cfg=cfg, stream=_stream(stream))
+                        softmax_scale, d_rope_cs=cp, cfg=cfg, stream=_stream(stream))
     return out
 
 
@@ -121,15 +140,18 @@ def packed_mmrope_attention(segments, q, k, v, perm=None, theta=10000.0, section
     """The whole path on one packed sequence: coords -> rotate Q, K -> attention.
 
     q, k, v: [N, H, 128] bf16 on the GPU (unrotated).  Returns O [N, H, 128].
-    fused_q_rope: rotate only K beforehand and Q inside the attention kernel.
+    fused_q_rope: rotate only K beforehand and Q inside the attention kernel
+    (from the rows' rotary table).
     """
     n = q.shape[-3]
     coords = build_coords(segments, n, perm, stream=stream)
     if fused_q_rope:
+        cs = rope_cos_sin(coords, theta=theta, sections=sections, pair_layout=pair_layout, freq_rule=freq_rule,
+                          stream=stream)
         _, kr = mmrope_qk(None, k, coords, theta=theta, sections=sections, pair_layout=pair_layout,
                           stream=stream, freq_rule=freq_rule)
         return packed_attention(q, kr, v, out=out, lse=lse, softmax_scale=softmax_scale, stream=stream,
-                                coords=coords, theta=theta, sections=sections, pair_layout=pair_layout,
+                                rope_cs=cs, theta=theta, sections=sections, pair_layout=pair_layout,
                                 freq_rule=freq_rule)
     qr, kr = mmrope_qk(q, k, coords, theta=theta, sections=sections, pair_layout=pair_layout, stream=stream,
                        freq_rule=freq_rule)

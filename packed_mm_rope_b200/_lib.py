@@ -19,7 +19,7 @@ H3_SEG_TEXT, H3_SEG_VIDEO, H3_SEG_AUDIO = 0, 1, 2
 H3_FLAG_TEXT_T_ONLY, H3_FLAG_AUDIO_CHANNEL_H, H3_FLAG_VIDEO_CANVAS = 1, 2, 4
 H3_MAX_SEGMENTS = 64
 
-EXPORTED = ("h3_status_str", "h3_version", "h3_build_coords", "h3_mmrope_qk",
+EXPORTED = ("h3_status_str", "h3_version", "h3_build_coords", "h3_mmrope_qk", "h3_rope_cos_sin",
             "h3_packed_attention", "h3_check_device_error", "h3_set_wait_limit_ns",
             "h3_host_workspace_bytes", "h3_packed_mmrope_attention_host",
             "h3_packed_mmrope_attention_host_noalloc", "h3_adaln_modulate", "h3_init", "h3_shutdown")
@@ -63,6 +63,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.h3_build_coords.argtypes = [ctypes.POINTER(h3_segment), I32, P, I64, P, P]
     lib.h3_mmrope_qk.restype = I32
     lib.h3_mmrope_qk.argtypes = [P, P, P, P, P, I64, I32, I64, ctypes.POINTER(h3_rope_cfg), P]
+    lib.h3_rope_cos_sin.restype = I32
+    lib.h3_rope_cos_sin.argtypes = [P, I64, ctypes.POINTER(h3_rope_cfg), P, P]
     lib.h3_packed_attention.restype = I32
     lib.h3_packed_attention.argtypes = [P, P, P, P, P, P, ctypes.POINTER(h3_rope_cfg), I32, I64, I32, I32,
                                         I64, F32, P]
@@ -124,11 +126,16 @@ def h3_mmrope_qk(d_q: int, d_k: int, d_q_out: int, d_k_out: int, d_coords: int, 
                                n_rows, n_heads, row_stride, ctypes.byref(cfg), stream or None), "h3_mmrope_qk")
 
 
+def h3_rope_cos_sin(d_coords: int, n_rows: int, cfg: h3_rope_cfg, d_cs: int, stream: int = 0) -> None:
+    _check(load().h3_rope_cos_sin(d_coords or None, n_rows, ctypes.byref(cfg), d_cs or None, stream or None),
+           "h3_rope_cos_sin")
+
+
 def h3_packed_attention(d_q: int, d_k: int, d_v: int, d_o: int, d_lse: int, batch: int, n_rows: int,
                         n_heads: int, row_stride: int, softmax_scale: float = 0.0, head_dim: int = 128,
-                        d_coords: int = 0, cfg: h3_rope_cfg | None = None, stream: int = 0) -> None:
+                        d_rope_cs: int = 0, cfg: h3_rope_cfg | None = None, stream: int = 0) -> None:
     _check(load().h3_packed_attention(d_q or None, d_k or None, d_v or None, d_o or None, d_lse or None,
-                                      d_coords or None, ctypes.byref(cfg) if cfg is not None else None,
+                                      d_rope_cs or None, ctypes.byref(cfg) if cfg is not None else None,
                                       batch, n_rows, n_heads, head_dim, row_stride, softmax_scale,
                                       stream or None), "h3_packed_attention")
 

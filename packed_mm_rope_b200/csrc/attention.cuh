@@ -104,10 +104,9 @@ struct Params {
   unsigned long long wait_limit_ns;
   unsigned long long drain_limit_ns;
   int err_slot;                   // error word of the launching stream
-  // fused RoPE on Q (coords == null: Q arrives rotated)
-  const float* coords;            // [B][N][3]
+  // fused RoPE on Q (rope_cs == null: Q arrives rotated)
+  const float2* rope_cs;          // [B][N][64] (cos, sin) per rotary pair
   int rope_layout;                // 0 adjacent pairs, 1 half-split
-  RopeTable rope;
 };
 
 // 2^(x*sl2 - m) for 64 logits: bf16 pairs and their sum.  Two logits per
@@ -158,7 +157,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   auto bar_o_full = [&](int i) { return bar0 + 8u * (10 + 2 * KV_STAGES + i); };
   const uint32_t bar_mma_done = bar0 + 8u * (12 + 2 * KV_STAGES);
   auto bar_q_ready = [&](int i) { return bar0 + 8u * (13 + 2 * KV_STAGES + i); };
-  const bool fused_rope = p.coords != nullptr;
+  const bool fused_rope = p.rope_cs != nullptr;
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gbase + SMEM_MISC);
   volatile uint32_t* const abort_flag = reinterpret_cast<volatile uint32_t*>(gbase + SMEM_MISC + 4);
 
@@ -363,33 +362,37 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     };
 
     // Fused RoPE: rotate this warpgroup's Q tile in shared memory, one thread
-    // per row, with the rope kernel's arithmetic (rope_cos_sin, rot2), then
-    // make the generic-proxy writes visible to the tensor core (async proxy).
+    // per row, with the (cos, sin) the rope kernel uses (read from the table)
+    // and its rot2 arithmetic, then make the generic-proxy writes visible to
+    // the tensor core (async proxy).
     if (fused_rope) {
       if (!warp_wait(bar_q_full(wg), 0, abort_flag, limit, eslot)) ok = false;
       const int row = q_row0 + wg * BM + row_in_tile;
       if (ok && row < p.n_rows) {
-        const float* crd = p.coords + (static_cast<long long>(batch) * p.n_rows + row) * 3;
-        const float c3[3] = {crd[0], crd[1], crd[2]};
+        const float4* cs4 = reinterpret_cast<const float4*>(p.rope_cs + (static_cast<long long>(batch) * p.n_rows + row) * 64);
         uint8_t* qrow = gbase + SMEM_Q + wg * TILE_BYTES + row_in_tile * 128;
         const int sw = row_in_tile & 7;           // 128-byte swizzle of this row
         auto chunk = [&](int c) {                 // logical 16-byte chunk c of 16
           return reinterpret_cast<uint4*>(qrow + (c >> 3) * HALF_BYTES + (((c & 7) ^ sw) << 4));
         };
         if (p.rope_layout == 0) {
-#pragma unroll 1
-          for (int c = 0; c < 16; ++c) {
-            float2 cs[4];
-#pragma unroll
-            for (int m = 0; m < 4; ++m) cs[m] = rope_cos_sin(p.rope, c3, 4 * c + m);
+#pragma unroll 4
+          for (int c = 0; c < 16; ++c) {          // pairs 4c .. 4c+3
+            const float4 a = __ldg(cs4 + 2 * c), b = __ldg(cs4 + 2 * c + 1);
+            const float2 cs[4] = {make_float2(a.x, a.y), make_float2(a.z, a.w), make_float2(b.x, b.y),
+                                  make_float2(b.z, b.w)};
             *chunk(c) = rotate_adjacent(*chunk(c), cs);
           }
         } else {
-#pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
+#pragma unroll 2
+          for (int c = 0; c < 8; ++c) {           // pairs 8c .. 8c+7
             float2 cs[8];
 #pragma unroll
-            for (int m = 0; m < 8; ++m) cs[m] = rope_cos_sin(p.rope, c3, 8 * c + m);
+            for (int m = 0; m < 4; ++m) {
+              const float4 a = __ldg(cs4 + 4 * c + m);
+              cs[2 * m] = make_float2(a.x, a.y);
+              cs[2 * m + 1] = make_float2(a.z, a.w);
+            }
             uint4 a = *chunk(c), b = *chunk(c + 8);
             rotate_half(a, b, cs);
             *chunk(c) = a;

@@ -97,16 +97,17 @@ EncodeTiledFn encode_tiled() {
 }
 
 // 3-D map over a bf16 [batch][n_rows][row_stride] tensor whose first
-// n_heads*128 columns are used; box = 64 columns x 128 rows, 128-byte swizzle.
+// n_heads*128 columns are used; box = 64 columns x box_rows rows, 128-byte
+// swizzle.
 bool make_qkv_map(CUtensorMap* map, const void* ptr, int32_t batch, int64_t n_rows, int32_t n_heads,
-                  int64_t row_stride) {
+                  int64_t row_stride, uint32_t box_rows) {
   EncodeTiledFn fn = encode_tiled();
   if (fn == nullptr) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(n_heads) * 128u, static_cast<cuuint64_t>(n_rows),
                               static_cast<cuuint64_t>(batch)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_stride) * 2u,
                                  static_cast<cuuint64_t>(row_stride) * 2u * static_cast<cuuint64_t>(n_rows)};
-  const cuuint32_t box[3] = {64u, 128u, 1u};
+  const cuuint32_t box[3] = {64u, box_rows, 1u};
   const cuuint32_t estride[3] = {1u, 1u, 1u};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
                   estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -254,15 +255,32 @@ h3_status h3_mmrope_qk(const void* d_q, const void* d_k, void* d_q_out, void* d_
   return cudaGetLastError() == cudaSuccess ? H3_OK : H3_ERR_CUDA;
 }
 
+h3_status h3_rope_cos_sin(const float* d_coords, int64_t n_rows, const h3_rope_cfg* cfg, float* d_cs,
+                          void* stream) {
+  if (n_rows < 0 || !valid_rope_cfg(cfg)) return H3_ERR_INVALID_ARG;
+  if (cfg->head_dim != 128) return H3_ERR_UNSUPPORTED;
+  if (n_rows == 0) return H3_OK;
+  if (!d_coords || !d_cs) return H3_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(d_cs) & 15u) != 0) return H3_ERR_UNSUPPORTED;
+  if (n_rows > (1ll << 40)) return H3_ERR_INVALID_ARG;
+  const h3::RopeTable tab = make_rope_table(cfg);
+  const long long need = (n_rows * 64 + 255) / 256;
+  const int grid = static_cast<int>(need < 16LL * sm_count() ? need : 16LL * sm_count());
+  h3::rope_cos_sin_kernel<<<grid, 256, 0, as_stream(stream)>>>(d_coords, n_rows, reinterpret_cast<float2*>(d_cs),
+                                                               tab);
+  return cudaGetLastError() == cudaSuccess ? H3_OK : H3_ERR_CUDA;
+}
+
 h3_status h3_packed_attention(const void* d_q, const void* d_k, const void* d_v, void* d_o, float* d_lse,
-                              const float* d_coords, const h3_rope_cfg* cfg, int32_t batch, int64_t n_rows,
+                              const float* d_rope_cs, const h3_rope_cfg* cfg, int32_t batch, int64_t n_rows,
                               int32_t n_heads, int32_t head_dim, int64_t row_stride, float softmax_scale,
                               void* stream) {
   if (batch < 1 || n_heads < 1 || n_rows < 0 || n_rows >= (1ll << 31)) return H3_ERR_INVALID_ARG;
   if (head_dim != 128) return H3_ERR_UNSUPPORTED;
-  if (d_coords != nullptr) {
+  if (d_rope_cs != nullptr) {
     if (!valid_rope_cfg(cfg)) return H3_ERR_INVALID_ARG;
     if (cfg->head_dim != 128) return H3_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(d_rope_cs) & 15u) != 0) return H3_ERR_UNSUPPORTED;
   }
   if (row_stride < static_cast<int64_t>(n_heads) * 128) return H3_ERR_INVALID_ARG;
   if (batch > 65535 || n_heads > 65535) return H3_ERR_INVALID_ARG;
@@ -272,9 +290,9 @@ h3_status h3_packed_attention(const void* d_q, const void* d_k, const void* d_v,
   if (row_stride % 8 != 0 || !aligned16(d_q) || !aligned16(d_k) || !aligned16(d_v) || !aligned16(d_o))
     return H3_ERR_UNSUPPORTED;
   CUtensorMap tq, tk, tv;
-  if (!make_qkv_map(&tq, d_q, batch, n_rows, n_heads, row_stride) ||
-      !make_qkv_map(&tk, d_k, batch, n_rows, n_heads, row_stride) ||
-      !make_qkv_map(&tv, d_v, batch, n_rows, n_heads, row_stride))
+  if (!make_qkv_map(&tq, d_q, batch, n_rows, n_heads, row_stride, 128) ||
+      !make_qkv_map(&tk, d_k, batch, n_rows, n_heads, row_stride, 128) ||
+      !make_qkv_map(&tv, d_v, batch, n_rows, n_heads, row_stride, 128))
     return H3_ERR_CUDA;
   if (device_state() == nullptr) return H3_ERR_CUDA;
 
@@ -291,10 +309,8 @@ h3_status h3_packed_attention(const void* d_q, const void* d_k, const void* d_v,
   p.wait_limit_ns = g_wait_limit_ns.load();
   p.drain_limit_ns = kDrainLimitNs;
   p.err_slot = error_slot(stream);
-  p.coords = d_coords;
-  p.rope_layout = d_coords ? cfg->pair_layout : 0;
-  if (d_coords) p.rope = make_rope_table(cfg);
-  else std::memset(&p.rope, 0, sizeof(p.rope));
+  p.rope_cs = reinterpret_cast<const float2*>(d_rope_cs);
+  p.rope_layout = d_rope_cs ? cfg->pair_layout : 0;
   const dim3 grid(static_cast<unsigned>((n_rows + 2 * h3::attn::BM - 1) / (2 * h3::attn::BM)),
                   static_cast<unsigned>(n_heads), static_cast<unsigned>(batch));
   h3::attn::attention_kernel<<<grid, h3::attn::THREADS, h3::attn::SMEM_BYTES, as_stream(stream)>>>(tq, tk, tv,

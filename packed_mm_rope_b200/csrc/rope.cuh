@@ -73,6 +73,17 @@ __device__ __forceinline__ void rotate_half(uint4& a, uint4& b, const float2* cs
   b = make_uint4(wb[0], wb[1], wb[2], wb[3]);
 }
 
+// The (cos, sin) of every rotary pair of every row, exactly as the rotation
+// uses them: one thread per (row, pair), consecutive threads writing
+// consecutive 8-byte entries of the [n_rows][64] table.
+__global__ void __launch_bounds__(256) rope_cos_sin_kernel(const float* __restrict__ coords, long long n_rows,
+                                                           float2* __restrict__ cs, const RopeTable tab) {
+  const long long n = n_rows * 64;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    cs[i] = rope_cos_sin(tab, coords + 3 * (i >> 6), static_cast<int>(i & 63));
+}
+
 // One warp per packed row.  A row of one tensor is n_heads x 16 chunks of 16
 // bytes; lane l handles the chunks (or, half-split, the chunk pairs) l, l + 32,
 // ...  Because 32 is a multiple of the chunks per head, a lane always meets the

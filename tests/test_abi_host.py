@@ -107,8 +107,8 @@ def test_attention_rejects_bad_arguments():
     assert _err(A, P, P, P, P, 0, 1, 10, 1, 132) == h3.H3_ERR_UNSUPPORTED
     assert _err(A, P, P, P + 4, P, 0, 1, 10, 1, 128) == h3.H3_ERR_UNSUPPORTED
     assert _err(A, P, P, 0, P, 0, 1, 10, 1, 128) == h3.H3_ERR_INVALID_ARG
-    assert _err(A, P, P, P, P, 0, 1, 10, 1, 128, d_coords=P) == h3.H3_ERR_INVALID_ARG     # no cfg
-    assert _err(A, P, P, P, P, 0, 1, 10, 1, 128, d_coords=P,
+    assert _err(A, P, P, P, P, 0, 1, 10, 1, 128, d_rope_cs=P) == h3.H3_ERR_INVALID_ARG     # no cfg
+    assert _err(A, P, P, P, P, 0, 1, 10, 1, 128, d_rope_cs=P,
                 cfg=h3.rope_cfg(sections=(32, 48, 40))) == h3.H3_ERR_INVALID_ARG
     assert _err(A, P, P, P, P, 0, 1, 10, 1, 128, softmax_scale=float("nan")) == h3.H3_ERR_INVALID_ARG
 
@@ -138,3 +138,16 @@ def test_host_calls_check_the_segment_table_before_queuing_anything():
     # too many head chunks is also refused up front
     assert _err(h3.h3_packed_mmrope_attention_host, [W.text(4)], 0, P, P, P, P, WORK, 4, 65, cfg, 1) == \
         h3.H3_ERR_UNSUPPORTED
+
+
+def test_rope_table_rejects_bad_arguments():
+    P = 0x10000
+    T = h3.h3_rope_cos_sin
+    h3.h3_rope_cos_sin(0, 0, h3.rope_cfg(), 0)                                     # empty: no-op
+    assert _err(T, P, 4, h3.rope_cfg(sections=(32, 48, 46)), P) == h3.H3_ERR_INVALID_ARG
+    assert _err(T, 0, 4, h3.rope_cfg(), P) == h3.H3_ERR_INVALID_ARG
+    assert _err(T, P, 4, h3.rope_cfg(), 0) == h3.H3_ERR_INVALID_ARG
+    assert _err(T, P, 4, h3.rope_cfg(), P + 8) == h3.H3_ERR_UNSUPPORTED             # table not 16-byte aligned
+    assert _err(T, P, 4, h3.rope_cfg(head_dim=256, sections=(64, 96, 96)), P) == h3.H3_ERR_UNSUPPORTED
+    A = h3.h3_packed_attention
+    assert _err(A, P, P, P, P, 0, 1, 10, 1, 128, d_rope_cs=P + 8, cfg=h3.rope_cfg()) == h3.H3_ERR_UNSUPPORTED

@@ -307,6 +307,27 @@ def test_fused_q_rope_is_identical_to_rotating_first(h3, cfg, layout, rule):
     check_attention(bf16_bits_to_f64(from_dev_bf16(o_fus)), ref, f"fused {wl.name}")
 
 
+@pytest.mark.parametrize("cfg,rule", [(0, 0), (4, 0), (1, 1)])
+def test_rope_table_matches_the_oracle_angles(h3, cfg, rule):
+    # h3_rope_cos_sin: (cos, sin) of the angle of the fp32 coordinate, each
+    # rounded to fp32.  The oracle evaluates the same angle in fp64 with
+    # numpy; the two fp64 values differ by a few fp64 ulps at most, so the
+    # fp32 results agree except, rarely, by one fp32 ulp at a rounding boundary.
+    # Workload 4 holds the largest |t| (reference audio down to about -6,000).
+    wl = W.workload(cfg)
+    perm = W.permutation(wl)
+    coords = h3.build_coords(wl.segments, wl.n_rows, _perm_dev(perm))
+    got = h3.rope_cos_sin(coords, theta=wl.theta, sections=wl.sections, freq_rule=rule).cpu().numpy()
+    _sync_ok(h3)
+    num, den = ocoords.packed_coords(wl.segments, perm)
+    ang = orope.angles(ocoords.to_f32(num, den).astype(np.float64), wl.theta, wl.sections, rule)
+    want = np.stack([np.cos(ang), np.sin(ang)], axis=-1).astype(np.float32)
+    assert got.shape == want.shape == (wl.n_rows, 64, 2)
+    ulp = np.spacing(np.abs(want).astype(np.float32))
+    assert (np.abs(got.astype(np.float64) - want) <= ulp).all()
+    assert (got == want).mean() > 0.9999
+
+
 def test_rope_k_only_leaves_q_alone(h3):
     wl = W.workload(0)
     perm = W.permutation(wl)
@@ -329,7 +350,7 @@ def test_fused_q_rope_ragged_batch(h3):
     dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
     qr, kr = h3.mmrope_qk(dq, dk, coords)
     o_sep = h3.packed_attention(qr, kr, dv)
-    o_fus = h3.packed_attention(dq, kr, dv, coords=coords)
+    o_fus = h3.packed_attention(dq, kr, dv, rope_cs=h3.rope_cos_sin(coords))
     _sync_ok(h3)
     assert torch.equal(o_sep, o_fus)
 
