@@ -9,8 +9,7 @@ locally per head; a second all-to-all returns each rank's rows.
 
 Heads and rows are split as evenly as possible (42 heads over 4 ranks:
 11, 11, 10, 10).  The exchanges are torch.distributed all-to-alls (NCCL on
-GPUs); the per-head work runs in the library's kernels.  ``local_attention``
-can be replaced only to test the exchange logic on CPU processes.
+GPUs); the per-head work runs in the library's kernels.
 """
 from __future__ import annotations
 
@@ -57,7 +56,7 @@ def _library_attention(segments, perm, q, k, v, theta, sections, pair_layout):
 
 
 def ulysses_packed_mmrope_attention(segments, q_shard, k_shard, v_shard, perm=None, group=None,
-                                    theta: float = 10000.0, sections=(32, 48, 48), pair_layout: int = 0,
+                                    theta: float = 10000.0, sections=(32, 48, 48), pair_layout: int = 0, *,
                                     local_attention: Optional[Callable] = None):
     """Packed MM-RoPE attention with rows sharded over the ranks of ``group``.
 
@@ -65,6 +64,10 @@ def ulysses_packed_mmrope_attention(segments, q_shard, k_shard, v_shard, perm=No
     even split of the packed sequence (rank order = row order).  ``perm``:
     the packed-row permutation of the whole sequence (as for
     h3_build_coords) or None.  Returns this rank's output rows [n_r, H, 128].
+
+    ``local_attention`` (keyword only) replaces the library's per-head step;
+    it exists so the exchange logic can be tested on CPU processes, where
+    the library's kernels cannot run.  Leave it unset.
     """
     import torch
     import torch.distributed as dist
