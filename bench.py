@@ -340,12 +340,16 @@ def profiled_traffic(wl):
     """
     import hashlib
     path = os.path.join(ROOT, "profiles", "attention_traffic.json")
-    src = os.path.join(ROOT, "packed_mm_rope_b200", "csrc", "attention.cuh")
+    # the attention kernel is built from these three files
+    srcs = [os.path.join(ROOT, "packed_mm_rope_b200", "csrc", n) for n in ("attention.cuh", "common.cuh", "rope.cuh")]
     try:
         with open(path) as f:
             d = json.load(f)
-        with open(src, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        h = hashlib.sha256()
+        for src in srcs:
+            with open(src, "rb") as f:
+                h.update(f.read())
+        sha = h.hexdigest()[:16]
         if d.get("n_rows") == wl.n_rows and d.get("heads") == wl.heads and d.get("source_sha256_16") == sha:
             return d.get("dram_bytes_per_launch")
     except (OSError, ValueError):

@@ -261,13 +261,17 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                  IDESC_O, (acc || kk > 0) ? 1u : 0u);
         }
       };
-      // P_i(j) in two halves; the first half's completion is announced on pva_done
-      auto issue_pv_tile = [&](int i, int vs, int j) -> bool {
+      // P_i(j) in two halves; the first half's completion is announced on pva_done.
+      // x (non-zero): a barrier the caller needs next, polled together with the
+      // second half of P so that the two polls' latencies overlap
+      auto issue_pv_tile = [&](int i, int vs, int j, uint32_t x, uint32_t x_par) -> bool {
         if (!mma_wait(bar_p_full(i, 0), j & 1, abort_flag, limit, eslot)) return false;
         tc_fence_after();
         issue_pv(i, vs, 0, j > 0);
         tc_commit(bar_pva_done(i));
-        if (!mma_wait(bar_p_full(i, 1), j & 1, abort_flag, limit, eslot)) return false;
+        if (x != 0u ? !mbar_spin2_bounded(bar_p_full(i, 1), j & 1, x, x_par, abort_flag, limit, eslot)
+                    : !mma_wait(bar_p_full(i, 1), j & 1, abort_flag, limit, eslot))
+          return false;
         tc_fence_after();
         issue_pv(i, vs, 1, true);
         return true;
@@ -293,16 +297,17 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int kidx = 2 * j + 2, ks = kidx % KV_STAGES;
         const bool more = j + 1 < nkv;
         if (!mma_wait(bar_kv_full(vs), (vidx / KV_STAGES) & 1, abort_flag, limit, eslot)) break;
-        if (!issue_pv_tile(0, vs, j)) break;
+        // K(j + 1) is waited for together with the second half of P0(j): the chain
+        // P0(j) -> P.V -> S0(j + 1) -> softmax pays one poll instead of two
+        if (!issue_pv_tile(0, vs, j, more ? bar_kv_full(ks) : 0u, (kidx / KV_STAGES) & 1)) break;
         if (more) {
-          if (!mma_wait(bar_kv_full(ks), (kidx / KV_STAGES) & 1, abort_flag, limit, eslot)) break;
           tc_fence_after();
           issue_s(0, ks);
           tc_commit(bar_s_full(0));
         } else {
           tc_commit(bar_o_full(0));
         }
-        if (!issue_pv_tile(1, vs, j)) break;
+        if (!issue_pv_tile(1, vs, j, 0u, 0u)) break;
         tc_commit(bar_kv_empty(vs));
         if (more) {
           issue_s(1, ks);
