@@ -7,34 +7,44 @@
 // head), no mask, every row attends to every row.
 //
 // Design (one CTA per 256 query rows of one head, one CTA per SM):
-//   warps 0-3   softmax warpgroup for query tile 0 (rows   0..127)
-//   warps 4-7   softmax warpgroup for query tile 1 (rows 128..255)
-//   warp  8     TMA producer: Q tiles once, then K_j, V_j into a ring
-//   warp  9     TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 0-7   softmax for query tile 0 (rows   0..127)
+//   warps 8-15  softmax for query tile 1 (rows 128..255)
+//   warp  16    TMA producer: Q tiles once, then K_j, V_j into a ring
+//   warp  17    TMEM allocator and single-thread tcgen05.mma issuer
 // Tensor memory (512 columns x 128 lanes, fp32):
 //   [  0,128)  S0 = Q0 K_j^T    (P0 = bf16 softmax numerators aliased on
 //   [128,256)  S1 = Q1 K_j^T     its first 64 columns, two per column)
 //   [256,384)  O0 accumulator   [384,512) O1 accumulator
 // Per KV tile j the issuer runs  PV0(j), S0(j+1), PV1(j), S1(j+1): while one
-// warpgroup exponentiates its S tile the tensor core works on the other.  Each
-// P tile is released in two 64-key halves with their own barriers, so the
-// first half of P.V runs while the second half is still being exponentiated.
+// query tile's warps exponentiate their S tile the tensor core works on the
+// other.  Each P tile is released in two 64-key halves with their own
+// barriers, so the first half of P.V runs while the second half is still being
+// exponentiated.  The issuing thread polls K(j+1) together with the second
+// half of P0(j): one barrier poll whose result is branched on costs it ~160
+// cycles, and this one sits on the chain P0(j) -> P.V -> S0(j+1) -> softmax.
 //
-// Softmax (one thread = one query row, the row lives in one TMEM lane):
-// logits are handled in log2 units (x = s * scale * log2 e).  Numerators are
-// 2^(x - m) against a running reference m that is only raised when a 64-key
-// half would overflow the headroom: the half's numerators are computed first
-// (speculatively, against the current m) and kept unless their sum exceeds
-// 2^64.  Then the half's true maximum is taken, O (in TMEM) and the row sum
-// are multiplied by 2^(m_old - m_new), and the half is recomputed.  Any m
+// Softmax: four threads per query row.  Warp w of a query tile reads the 16
+// TMEM lanes 32 (w % 4) + 16 ((w / 4) % 2) + [0, 16) with the 16x256b shape,
+// so thread (t0 = lane % 4, t1 = lane / 4) holds rows t1 and t1 + 8 of those
+// lanes and, of every 8-column block, columns 2 t0 and 2 t0 + 1; the four
+// threads of a row (a quad) together hold its 128 keys.  Four warps per
+// sub-partition hide each other's TMEM and barrier latencies (one thread per
+// row leaves two).  Logits are handled in log2 units (x = s * scale * log2 e).
+// Numerators are 2^(x - m) against a running reference m per row that is only
+// raised when a thread's share of a 64-key half would overflow the headroom:
+// the half's numerators are computed first (speculatively, against the current
+// m) and kept unless a share exceeds 2^62 (four shares stay below 2^64).  Then
+// the quad takes the half's true maximum by shuffles, O (in TMEM) and the row
+// sums are multiplied by 2^(m_old - m_new), and the half is recomputed.  Any m
 // gives the same quotient O / l; the limit only keeps numerators, sums and O
 // far from fp32/bf16 overflow.  In practice m is set by the first half-tile
 // and never moves again, so the hot loop has no max reduction at all: one
 // packed fp32x2 FMA, two MUFU ex2, one packed add and one bf16x2 conversion per
 // pair of logits.  The S tile of step j+1 is only issued after PV(j), so when
-// a warpgroup sees S(j) complete, O already holds PV(j-1) and a rescale for
-// the first half can be applied in place; a rescale for the second half first
-// waits for the first half of PV(j) to land (pva_done).
+// a warp sees S(j) complete, O already holds PV(j-1) and a rescale for the
+// first half can be applied in place; a rescale for the second half first
+// waits for the first half of PV(j) to land (pva_done).  Each thread keeps its
+// share of the row sums; the quad adds them once, in the epilogue.
 //
 // Shared memory (1024-byte aligned): Q0, Q1 (32 KB each) and a ring of
 // KV_STAGES 32 KB slots; every 128 x 128 bf16 tile is two 128-row x 64-column
@@ -56,10 +66,9 @@ constexpr int BM = 128;          // query rows per tile (MMA M)
 constexpr int BN = 128;          // key rows per tile  (S MMA N, PV MMA K)
 constexpr int HD = 128;          // head dim
 constexpr int KV_STAGES = 4;     // K/V ring slots of 32 KB
-constexpr int THREADS = 320;
+constexpr int THREADS = 576;   // 16 softmax warps, producer, MMA issuer
 constexpr uint32_t TILE_BYTES = BM * HD * 2;     // 32768
 constexpr uint32_t HALF_BYTES = TILE_BYTES / 2;  // 16384
-constexpr float SUM_LIMIT = 18446744073709551616.0f;   // 2^64
 
 constexpr uint32_t SMEM_Q = 0;
 constexpr uint32_t SMEM_KV = 2 * TILE_BYTES;
@@ -109,36 +118,6 @@ struct Params {
   int rope_layout;                // 0 adjacent pairs, 1 half-split
 };
 
-// 2^(x*sl2 - m) for 64 logits: bf16 pairs and their sum.  Two logits per
-// packed fp32x2 FMA and add (Blackwell f32x2 arithmetic) keep the instruction
-// count per element at 2.5: the softmax warps are issue-bound, not MUFU-bound.
-__device__ __forceinline__ void exp_half(const float (&x)[64], float sl2, float m, uint32_t (&pk)[32],
-                                         float& ls) {
-  const float2 c2 = make_float2(sl2, sl2), mm = make_float2(-m, -m);
-  float2 acc[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
-#pragma unroll
-  for (int c = 0; c < 32; ++c) {
-    const float2 y = __ffma2_rn(make_float2(x[2 * c], x[2 * c + 1]), c2, mm);
-    const float p0 = ex2_approx(y.x), p1 = ex2_approx(y.y);
-    acc[c & 3] = __fadd2_rn(acc[c & 3], make_float2(p0, p1));
-    pk[c] = pack_bf16x2(p0, p1);
-  }
-  const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-  ls = t.x + t.y;
-}
-
-// Raw maximum of 64 logits (only on the rare rescale path).
-__device__ __forceinline__ float max64(const float (&x)[64]) {
-  float ma[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) ma[i] = x[i];
-#pragma unroll
-  for (int c = 8; c < 64; ++c) ma[c & 7] = fmaxf(ma[c & 7], x[c]);
-  return fmaxf(fmaxf(fmaxf(ma[0], ma[1]), fmaxf(ma[2], ma[3])), fmaxf(fmaxf(ma[4], ma[5]), fmaxf(ma[6], ma[7])));
-}
-
 __global__ void __launch_bounds__(THREADS, 1)
 attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -174,8 +153,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_q_full(i), 1);
       mbar_init(bar_s_full(i), 1);
-      mbar_init(bar_p_full(i, 0), 128);
-      mbar_init(bar_p_full(i, 1), 128);
+      mbar_init(bar_p_full(i, 0), 8);    // one arrival per softmax warp of the tile
+      mbar_init(bar_p_full(i, 1), 8);
       mbar_init(bar_pva_done(i), 1);
       mbar_init(bar_o_full(i), 1);
     }
@@ -184,16 +163,16 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       mbar_init(bar_kv_empty(s), 1);
     }
     mbar_init(bar_mma_done, 1);
-    mbar_init(bar_q_ready(0), 128);
-    mbar_init(bar_q_ready(1), 128);
+    mbar_init(bar_q_ready(0), 8);
+    mbar_init(bar_q_ready(1), 8);
     *abort_flag = 0u;
     mbar_fence_init();
   }
-  if (warp == 9) {
+  if (warp == 17) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == 16 && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
@@ -203,7 +182,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == 16) {
     // ------------------------------------------------------------ TMA ----
     if (lane == 0) {
       const int col0 = head * HD;
@@ -234,7 +213,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mbar_wait_bounded(bar_kv_full(idx % KV_STAGES), (idx / KV_STAGES) & 1, &never,
                           p.drain_limit_ns, eslot);
     }
-  } else if (warp == 9) {
+  } else if (warp == 17) {
     // ------------------------------------------------------------ MMA ----
     if (lane == 0) {
       auto q_addr = [&](int i) { return base + SMEM_Q + i * TILE_BYTES; };
@@ -324,54 +303,129 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   } else {
     // -------------------------------------------------------- softmax ----
-    const int wg = warp >> 2;                      // query tile 0 or 1
-    const int row_in_tile = threadIdx.x & 127;     // == TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t t_s = tmem + lane_base + TMEM_S0 + wg * 128;
-    const uint32_t t_o = tmem + lane_base + TMEM_O0 + wg * 128;
+    // Eight warps per query tile, four threads per row: warp w reads the 16
+    // TMEM lanes 32 (w % 4) + 16 ((w / 4) % 2) + [0, 16) with the 16x256b
+    // shape, so thread (t0 = lane % 4, t1 = lane / 4) holds rows t1 and t1 + 8
+    // of that group and, of every 8-column block, columns 2 t0 and 2 t0 + 1.
+    // The four threads of a row agree on its reference through shuffles.
+    const int wg = warp >> 3;                      // query tile 0 or 1
+    const int t0 = lane & 3, t1 = lane >> 2;
+    const int lane16 = 32 * (warp & 3) + 16 * ((warp >> 2) & 1);
+    const uint32_t lb = static_cast<uint32_t>(lane16) << 16;
+    const uint32_t t_s = tmem + lb + TMEM_S0 + wg * 128;
+    const uint32_t t_o = tmem + lb + TMEM_O0 + wg * 128;
     const float sl2 = p.scale_log2;
     const int tail = p.n_rows - (nkv - 1) * BN;    // valid keys in the last tile (1..128)
-    float m_used = -INFINITY;                      // log2 units
-    float l_sum = 0.f;
+    const int row_a = q_row0 + wg * BM + lane16 + t1;
+    const int row_b = row_a + 8;
+    float m_a = -INFINITY, m_b = -INFINITY;        // log2 units, identical in a row's 4 threads
+    float l_a = 0.f, l_b = 0.f;                    // this thread's share of the row sums
     bool ok = true;
+    constexpr float PART_LIMIT = 4611686018427387904.0f;   // 2^62: four shares stay below 2^64
 
-    // registers of two TMEM chunks -> 64 logits; keys past the end -> -inf
-    auto to_logits = [&](const uint32_t (&r)[2][32], int col0, bool last, float (&x)[64]) {
+    auto quad_max = [](float v) {
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+      return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+    };
+    auto quad_or = [](bool v) {
+      int x = v ? 1 : 0;
+      x |= __shfl_xor_sync(0xffffffffu, x, 1);
+      x |= __shfl_xor_sync(0xffffffffu, x, 2);
+      return x != 0;
+    };
+    // logits of 64 keys starting at key c0 of the tile (registers as loaded);
+    // keys past the end -> -inf
+    auto to_logits = [&](const uint32_t (&r)[32], int c0, bool last, float (&x)[32]) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(r[c >> 5][c & 31]);
+      for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(r[e]);
       if (last && tail < BN) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (col0 + c >= tail) x[c] = -INFINITY;
+        for (int e = 0; e < 32; ++e) {
+          const int key = c0 + 8 * (e >> 2) + 2 * t0 + (e & 1);
+          if (key >= tail) x[e] = -INFINITY;
+        }
       }
     };
-    // O *= f for this warp's rows (warp-collective TMEM round trip)
-    auto rescale_o = [&](float f) {
+    // numerators of the 16 keys of each row: bf16 pairs (register order of the
+    // 16x128b store) and this thread's sums
+    auto exps = [&](const float (&x)[32], uint32_t (&pk)[16], float& sa, float& sb) {
+      const float2 c2 = make_float2(sl2, sl2);
+      const float2 ma = make_float2(-m_a, -m_a), mb = make_float2(-m_b, -m_b);
+      float2 acc_a = make_float2(0.f, 0.f), acc_b = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float2 ya = __ffma2_rn(make_float2(x[4 * q], x[4 * q + 1]), c2, ma);
+        const float2 yb = __ffma2_rn(make_float2(x[4 * q + 2], x[4 * q + 3]), c2, mb);
+        const float pa0 = ex2_approx(ya.x), pa1 = ex2_approx(ya.y);
+        const float pb0 = ex2_approx(yb.x), pb1 = ex2_approx(yb.y);
+        acc_a = __fadd2_rn(acc_a, make_float2(pa0, pa1));
+        acc_b = __fadd2_rn(acc_b, make_float2(pb0, pb1));
+        pk[2 * q] = pack_bf16x2(pa0, pa1);
+        pk[2 * q + 1] = pack_bf16x2(pb0, pb1);
+      }
+      sa = acc_a.x + acc_a.y;
+      sb = acc_b.x + acc_b.y;
+    };
+    // O *= f per row for this warp's lanes (warp-collective TMEM round trip)
+    auto rescale_o = [&](float fa, float fb) {
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int h = 0; h < 2; ++h) {
         uint32_t o[32];
-        tmem_ld32(t_o + 32 * c, o);
+        tmem_ld16x256(t_o + 64 * h, o);
         tmem_wait_ld(o);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-        tmem_st32(t_o + 32 * c, o);
+        for (int e = 0; e < 32; ++e)
+          o[e] = __float_as_uint(__uint_as_float(o[e]) * (((e >> 1) & 1) ? fb : fa));
+        tmem_st16x256(t_o + 64 * h, o);
       }
     };
-    // Publish 64 keys of P (32 TMEM columns, aliasing the S columns already read).
-    auto store_p = [&](int half, const uint32_t (&pk)[32]) {
+    // the rare path: raise the reference of the rows whose shares need it
+    // (all rows on the first half of the first tile); returns (fa, fb)
+    auto new_reference = [&](const float (&x)[32], bool first, float sa, float sb, float& fa, float& fb) {
+      const bool na = quad_or(first || !(sa <= PART_LIMIT));
+      const bool nb = quad_or(first || !(sb <= PART_LIMIT));
+      float xa = -INFINITY, xb = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        xa = fmaxf(xa, fmaxf(x[4 * q], x[4 * q + 1]));
+        xb = fmaxf(xb, fmaxf(x[4 * q + 2], x[4 * q + 3]));
+      }
+      xa = quad_max(xa);
+      xb = quad_max(xb);
+      fa = 1.f;
+      fb = 1.f;
+      if (na) {
+        const float mn = fmaxf(m_a, xa * sl2);
+        fa = first ? 0.f : ex2_approx(m_a - mn);
+        m_a = mn;
+        l_a *= fa;
+      }
+      if (nb) {
+        const float mn = fmaxf(m_b, xb * sl2);
+        fb = first ? 0.f : ex2_approx(m_b - mn);
+        m_b = mn;
+        l_b *= fb;
+      }
+    };
+    // Publish 64 keys of P (32 TMEM columns at c0 / 2, aliasing S columns
+    // already read): every lane's store lands and is fenced, then one arrival.
+    auto store_p = [&](int half, const uint32_t (&pk)[16]) {
       __syncwarp();
-      tmem_st32(t_s + 32 * half, pk);
+      tmem_st16x128(t_s + 32 * half, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_p_full(wg, half));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_p_full(wg, half));
     };
 
-    // Fused RoPE: rotate this warpgroup's Q tile in shared memory, one thread
-    // per row, with the (cos, sin) the rope kernel uses (read from the table)
-    // and its rot2 arithmetic, then make the generic-proxy writes visible to
-    // the tensor core (async proxy).
+    // Fused RoPE: rotate this tile's Q rows in shared memory, two threads per
+    // row (each 8 of the 16 chunks), with the (cos, sin) the rope kernel uses
+    // (read from the table) and its rot2 arithmetic, then make the
+    // generic-proxy writes visible to the tensor core (async proxy).
     if (fused_rope) {
       if (!warp_wait(bar_q_full(wg), 0, abort_flag, limit, eslot)) ok = false;
+      const int tid = (warp & 7) * 32 + lane;
+      const int row_in_tile = tid >> 1, part = tid & 1;
       const int row = q_row0 + wg * BM + row_in_tile;
       if (ok && row < p.n_rows) {
         const float4* cs4 = reinterpret_cast<const float4*>(p.rope_cs + (static_cast<long long>(batch) * p.n_rows + row) * 64);
@@ -382,7 +436,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         };
         if (p.rope_layout == 0) {
 #pragma unroll 4
-          for (int c = 0; c < 16; ++c) {          // pairs 4c .. 4c+3
+          for (int c = 8 * part; c < 8 * part + 8; ++c) {   // pairs 4c .. 4c+3
             const float4 a = __ldg(cs4 + 2 * c), b = __ldg(cs4 + 2 * c + 1);
             const float2 cs[4] = {make_float2(a.x, a.y), make_float2(a.z, a.w), make_float2(b.x, b.y),
                                   make_float2(b.z, b.w)};
@@ -390,7 +444,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           }
         } else {
 #pragma unroll 2
-          for (int c = 0; c < 8; ++c) {           // pairs 8c .. 8c+7
+          for (int c = 4 * part; c < 4 * part + 4; ++c) {   // pairs 8c .. 8c+7
             float2 cs[8];
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
@@ -406,109 +460,104 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(bar_q_ready(wg));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_q_ready(wg));
     }
 
-    for (int j = 0; j < nkv; ++j) {
+    for (int j = 0; ok && j < nkv; ++j) {
       if (!warp_wait(bar_s_full(wg), j & 1, abort_flag, limit, eslot)) { ok = false; break; }
       tc_fence_after();
       const bool last = j == nkv - 1;
-      float ls_a;
       {
         // ---- keys 0..63 ----
-        uint32_t ra[2][32];
-        tmem_ld32(t_s, ra[0]);
-        tmem_ld32(t_s + 32, ra[1]);
-        tmem_wait_ld(ra[0]);
-        tmem_wait_ld(ra[1]);
-        float xa[64];
-        to_logits(ra, 0, last, xa);
-        uint32_t pka[32];
-        exp_half(xa, sl2, m_used, pka, ls_a);         // speculative against m_used
-        const bool need = (j == 0) || !(ls_a <= SUM_LIMIT);
+        uint32_t r[32];
+        tmem_ld16x256(t_s, r);
+        tmem_wait_ld(r);
+        float x[32];
+        to_logits(r, 0, last, x);
+        uint32_t pk[16];
+        float sa, sb;
+        exps(x, pk, sa, sb);                        // speculative against the references
+        const bool need = (j == 0) || !(sa <= PART_LIMIT) || !(sb <= PART_LIMIT);
         if (__any_sync(0xffffffffu, need)) {
-          float f = 1.f;
-          if (need) {
-            const float m_new = fmaxf(m_used, max64(xa) * sl2);
-            f = (j == 0) ? 0.f : ex2_approx(m_used - m_new);
-            m_used = m_new;
-            l_sum *= f;
-          }
+          float fa, fb;
+          new_reference(x, j == 0, sa, sb, fa, fb);
           __syncwarp();
-          if (j > 0) rescale_o(f);      // O holds PV(j-1); PV(j) has not started
-          exp_half(xa, sl2, m_used, pka, ls_a);
+          if (j > 0) rescale_o(fa, fb);   // O holds PV(j-1); PV(j) has not started
+          exps(x, pk, sa, sb);
         }
-        l_sum += ls_a;
-        store_p(0, pka);
+        l_a += sa;
+        l_b += sb;
+        store_p(0, pk);
       }
       {
         // ---- keys 64..127 ----
-        uint32_t rb[2][32];
+        uint32_t r[32];
         __syncwarp();
-        tmem_ld32(t_s + 64, rb[0]);
-        tmem_ld32(t_s + 96, rb[1]);
-        tmem_wait_ld(rb[0]);
-        tmem_wait_ld(rb[1]);
-        float xb[64];
-        to_logits(rb, 64, last, xb);
-        uint32_t pkb[32];
-        float ls_b;
-        exp_half(xb, sl2, m_used, pkb, ls_b);
-        const bool need = !(ls_b <= SUM_LIMIT);
+        tmem_ld16x256(t_s + 64, r);
+        tmem_wait_ld(r);
+        float x[32];
+        to_logits(r, 64, last, x);
+        uint32_t pk[16];
+        float sa, sb;
+        exps(x, pk, sa, sb);
+        const bool need = !(sa <= PART_LIMIT) || !(sb <= PART_LIMIT);
         if (__any_sync(0xffffffffu, need)) {
           // the first half of PV(j) may be in flight: let it land, then rescale
-          // O (which now includes it) together with the running sum
+          // O (which now includes it) together with the running sums
           if (!warp_wait(bar_pva_done(wg), j & 1, abort_flag, limit, eslot)) { ok = false; break; }
           tc_fence_after();
-          float f = 1.f;
-          if (need) {
-            const float m_new = fmaxf(m_used, max64(xb) * sl2);
-            f = ex2_approx(m_used - m_new);
-            m_used = m_new;
-            l_sum *= f;
-          }
+          float fa, fb;
+          new_reference(x, false, sa, sb, fa, fb);
           __syncwarp();
-          rescale_o(f);
-          exp_half(xb, sl2, m_used, pkb, ls_b);
+          rescale_o(fa, fb);
+          exps(x, pk, sa, sb);
         }
-        l_sum += ls_b;
-        store_p(1, pkb);
+        l_a += sa;
+        l_b += sb;
+        store_p(1, pk);
       }
     }
 
     // epilogue: O / l -> bf16 -> global; optional log-sum-exp
     if (ok && warp_wait(bar_o_full(wg), 0, abort_flag, limit, eslot)) {
       tc_fence_after();
-      const int row = q_row0 + wg * BM + row_in_tile;
-      const float inv_l = 1.f / l_sum;
-      __nv_bfloat16* orow = p.o + batch * p.o_batch_stride + static_cast<long long>(row) * p.o_row_stride +
-                            head * HD;
+      // row sums over the four threads of each row
+      l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+      l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+      l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+      l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+      const float inv_a = 1.f / l_a, inv_b = 1.f / l_b;
+      __nv_bfloat16* orow_a = p.o + batch * p.o_batch_stride + static_cast<long long>(row_a) * p.o_row_stride + head * HD;
+      __nv_bfloat16* orow_b = orow_a + 8 * p.o_row_stride;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int h = 0; h < 2; ++h) {
         uint32_t o[32];
         __syncwarp();
-        tmem_ld32(t_o + 32 * c, o);
+        tmem_ld16x256(t_o + 64 * h, o);
         tmem_wait_ld(o);
-        uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-        if (row < p.n_rows) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+        for (int q = 0; q < 8; ++q) {
+          const int col = 64 * h + 8 * q + 2 * t0;
+          if (row_a < p.n_rows)
+            *reinterpret_cast<uint32_t*>(orow_a + col) =
+                pack_bf16x2(__uint_as_float(o[4 * q]) * inv_a, __uint_as_float(o[4 * q + 1]) * inv_a);
+          if (row_b < p.n_rows)
+            *reinterpret_cast<uint32_t*>(orow_b + col) =
+                pack_bf16x2(__uint_as_float(o[4 * q + 2]) * inv_b, __uint_as_float(o[4 * q + 3]) * inv_b);
         }
       }
-      if (p.lse != nullptr && row < p.n_rows) {
-        p.lse[(static_cast<long long>(batch) * p.n_heads + head) * p.n_rows + row] =
-            (m_used + __log2f(l_sum)) * 0.69314718055994530942f;
+      if (p.lse != nullptr && t0 == 0) {
+        float* lrow = p.lse + (static_cast<long long>(batch) * p.n_heads + head) * p.n_rows;
+        if (row_a < p.n_rows) lrow[row_a] = (m_a + __log2f(l_a)) * 0.69314718055994530942f;
+        if (row_b < p.n_rows) lrow[row_b] = (m_b + __log2f(l_b)) * 0.69314718055994530942f;
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 17) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
