@@ -19,9 +19,10 @@
 // query tile's warps exponentiate their S tile the tensor core works on the
 // other.  Each P tile is released in two 64-key halves with their own
 // barriers, so the first half of P.V runs while the second half is still being
-// exponentiated.  The issuing thread polls K(j+1) together with the second
-// half of P0(j): one barrier poll whose result is branched on costs it ~160
-// cycles, and this one sits on the chain P0(j) -> P.V -> S0(j+1) -> softmax.
+// exponentiated.  The issuing thread polls V(j) together with the first half of
+// P0(j) and K(j+1) together with its second half: one barrier poll whose result
+// is branched on costs it ~160 cycles, and the second pair sits on the chain
+// P0(j) -> P.V -> S0(j+1) -> softmax.
 //
 // Softmax: four threads per query row.  Warp w of a query tile reads the 16
 // TMEM lanes 32 (w % 4) + 16 ((w / 4) % 2) + [0, 16) with the 16x256b shape,
@@ -241,10 +242,13 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
       };
       // P_i(j) in two halves; the first half's completion is announced on pva_done.
-      // x (non-zero): a barrier the caller needs next, polled together with the
-      // second half of P so that the two polls' latencies overlap
-      auto issue_pv_tile = [&](int i, int vs, int j, uint32_t x, uint32_t x_par) -> bool {
-        if (!mma_wait(bar_p_full(i, 0), j & 1, abort_flag, limit, eslot)) return false;
+      // x / y (non-zero): a barrier the caller needs, polled together with the
+      // second / first half of P so that the two polls' latencies overlap
+      auto issue_pv_tile = [&](int i, int vs, int j, uint32_t x, uint32_t x_par, uint32_t y = 0u,
+                               uint32_t y_par = 0u) -> bool {
+        if (y != 0u ? !mbar_spin2_bounded(bar_p_full(i, 0), j & 1, y, y_par, abort_flag, limit, eslot)
+                    : !mma_wait(bar_p_full(i, 0), j & 1, abort_flag, limit, eslot))
+          return false;
         tc_fence_after();
         issue_pv(i, vs, 0, j > 0);
         tc_commit(bar_pva_done(i));
@@ -275,10 +279,11 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int vidx = 2 * j + 1, vs = vidx % KV_STAGES;
         const int kidx = 2 * j + 2, ks = kidx % KV_STAGES;
         const bool more = j + 1 < nkv;
-        if (!mma_wait(bar_kv_full(vs), (vidx / KV_STAGES) & 1, abort_flag, limit, eslot)) break;
-        // K(j + 1) is waited for together with the second half of P0(j): the chain
-        // P0(j) -> P.V -> S0(j + 1) -> softmax pays one poll instead of two
-        if (!issue_pv_tile(0, vs, j, more ? bar_kv_full(ks) : 0u, (kidx / KV_STAGES) & 1)) break;
+        // V(j) is waited for together with the first half of P0(j), K(j + 1)
+        // together with its second half
+        if (!issue_pv_tile(0, vs, j, more ? bar_kv_full(ks) : 0u, (kidx / KV_STAGES) & 1, bar_kv_full(vs),
+                           (vidx / KV_STAGES) & 1))
+          break;
         if (more) {
           tc_fence_after();
           issue_s(0, ks);
