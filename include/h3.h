@@ -318,7 +318,9 @@ uint64_t h3_host_workspace_bytes(int64_t n_rows, int32_t n_heads);
  *                     256-byte aligned, owned by the caller; contents undefined
  *                     after the call
  *   heads_per_chunk   0 = chosen by the library (chunks whose CTA count fills
- *                     whole waves of SMs), else 1..n_heads
+ *                     whole waves of SMs, the last few heads in halving
+ *                     chunks so that little work remains after the last copy
+ *                     in), else 1..n_heads heads per chunk
  *   cfg               host rotary configuration
  *   stream            work starts after everything already queued on `stream`;
  *                     the call returns once all work is queued, and `stream`

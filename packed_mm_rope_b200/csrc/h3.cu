@@ -417,6 +417,25 @@ int pick_heads_per_chunk(int64_t n_rows, int n_heads) {
   return best;
 }
 
+// Chunk sizes of the host pipeline: chunks of `hc` heads, and with `taper` the
+// last hc + (n_heads mod hc) heads in halving pieces (6 -> 3, 2, 1), so that the
+// attention and the copy out that remain after the last copy in are short.
+int plan_chunks(int n_heads, int hc, bool taper, int (&sizes)[64]) {
+  int n = 0, left = n_heads;
+  const int tail = taper ? std::min(n_heads, hc + n_heads % hc) : 0;
+  while (left > tail && n < 64) {
+    const int c = std::min(hc, left - tail > 0 ? left - tail : left);
+    sizes[n++] = c;
+    left -= c;
+  }
+  while (left > 0 && n < 64) {
+    const int c = (left + 1) / 2;
+    sizes[n++] = c;
+    left -= c;
+  }
+  return left == 0 ? n : -1;
+}
+
 }  // namespace
 
 extern "C" {
@@ -436,8 +455,9 @@ h3_status h3_packed_mmrope_attention_host(const h3_segment* segs, int32_t nseg, 
   if (n_rows >= (1ll << 31)) return H3_ERR_INVALID_ARG;
   if (d_work == nullptr || (reinterpret_cast<uintptr_t>(d_work) & 255u)) return H3_ERR_INVALID_ARG;
   const int hc = heads_per_chunk > 0 ? heads_per_chunk : pick_heads_per_chunk(n_rows, n_heads);
-  const int nchunks = (n_heads + hc - 1) / hc;
-  if (nchunks > 64) return H3_ERR_UNSUPPORTED;
+  int chunk_heads[64];
+  const int nchunks = plan_chunks(n_heads, hc, heads_per_chunk == 0, chunk_heads);
+  if (nchunks < 0) return H3_ERR_UNSUPPORTED;
   HostPipe* hp = host_pipe();
   if (hp == nullptr) return H3_ERR_CUDA;
   std::lock_guard<std::mutex> lock(hp->enqueue);
@@ -477,8 +497,8 @@ h3_status h3_packed_mmrope_attention_host(const h3_segment* segs, int32_t nseg, 
   st = h3_build_coords(segs, nseg, h_perm ? dperm : nullptr, n_rows, dcoords, stream);
   if (st != H3_OK) return fail(st);
 
-  for (int c = 0; c < nchunks; ++c) {
-    const int h0 = c * hc, nh = (h0 + hc <= n_heads) ? hc : n_heads - h0;
+  for (int c = 0, h0 = 0; c < nchunks; h0 += chunk_heads[c], ++c) {
+    const int nh = chunk_heads[c];
     const size_t off = static_cast<size_t>(h0) * 256u, width = static_cast<size_t>(nh) * 256u;
     for (int x = 0; x < 3; ++x) {
       const uint8_t* src = static_cast<const uint8_t*>(x == 0 ? h_q : x == 1 ? h_k : h_v) + off;
