@@ -67,7 +67,10 @@ constexpr int BM = 128;          // query rows per tile (MMA M)
 constexpr int BN = 128;          // key rows per tile  (S MMA N, PV MMA K)
 constexpr int HD = 128;          // head dim
 constexpr int KV_STAGES = 4;     // K/V ring slots of 32 KB
-constexpr int THREADS = 576;   // 16 softmax warps, producer, MMA issuer
+constexpr int SOFTMAX_WARPS = 16;                   // 8 per query tile, four threads per row
+constexpr int W_PROD = SOFTMAX_WARPS;                // TMA producer
+constexpr int W_MMA = SOFTMAX_WARPS + 1;             // TMEM allocator and MMA issuer
+constexpr int THREADS = 32 * (SOFTMAX_WARPS + 2);    // 576
 constexpr uint32_t TILE_BYTES = BM * HD * 2;     // 32768
 constexpr uint32_t HALF_BYTES = TILE_BYTES / 2;  // 16384
 
@@ -169,11 +172,11 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     *abort_flag = 0u;
     mbar_fence_init();
   }
-  if (warp == 17) {
+  if (warp == W_MMA) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 16 && lane == 0) {
+  if (warp == W_PROD && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
@@ -183,7 +186,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 16) {
+  if (warp == W_PROD) {
     // ------------------------------------------------------------ TMA ----
     if (lane == 0) {
       const int col0 = head * HD;
@@ -214,7 +217,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mbar_wait_bounded(bar_kv_full(idx % KV_STAGES), (idx / KV_STAGES) & 1, &never,
                           p.drain_limit_ns, eslot);
     }
-  } else if (warp == 17) {
+  } else if (warp == W_MMA) {
     // ------------------------------------------------------------ MMA ----
     if (lane == 0) {
       auto q_addr = [&](int i) { return base + SMEM_Q + i * TILE_BYTES; };
@@ -562,7 +565,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 17) {
+  if (warp == W_MMA) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
