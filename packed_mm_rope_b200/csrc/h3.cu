@@ -424,7 +424,7 @@ int plan_chunks(int n_heads, int hc, bool taper, int (&sizes)[64]) {
   int n = 0, left = n_heads;
   const int tail = taper ? std::min(n_heads, hc + n_heads % hc) : 0;
   while (left > tail && n < 64) {
-    const int c = std::min(hc, left - tail > 0 ? left - tail : left);
+    const int c = std::min(hc, left - tail);
     sizes[n++] = c;
     left -= c;
   }
