@@ -373,7 +373,7 @@ def cpu_threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(wl, q, k, v, perm, rows=384):
+def cpu_baseline(wl, q, k, v, perm, rows=768):
     import workload as W
     sample = np.sort(W.uniform01(wl.seed, 7, rows) * wl.n_rows).astype(np.int64)
     secs = oracle_sample(wl, q, k, v, perm, sample)
@@ -426,8 +426,8 @@ def main():
                     help="rotate only K in h3_mmrope_qk and Q inside h3_packed_attention (from h3_rope_cos_sin)")
     ap.add_argument("--adaln", action="store_true", help="also time h3_adaln_modulate on [N, H*128]")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=384,
-                    help="query rows of the timed oracle sample (384: about 10 s of host time at the worked example)")
+    ap.add_argument("--cpu-rows", type=int, default=768,
+                    help="query rows of the timed oracle sample (768: about 10 s of host time at the worked example)")
     ap.add_argument("--ref-rows", type=int, default=16, help="query rows per reference-arm step")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
