@@ -43,6 +43,25 @@ def test_host_path_equals_device_path(h3, cfg, chunk, pin):
         check_attention(got, ref, "host path")
 
 
+@pytest.mark.parametrize("heads", [42, 13])
+def test_host_path_tapered_chunks_many_heads(h3, heads):
+    # the small workload's rows with many heads: the library's own chunking
+    # (whole-wave chunks, then the last few heads in halving chunks) must give
+    # exactly the device-path result
+    import dataclasses
+    wl = dataclasses.replace(W.workload(1), heads=heads)
+    q, k, v = W.qkv_bf16(wl)
+    perm = W.permutation(wl)
+    dperm = None if perm is None else torch.from_numpy(perm.astype(np.int32)).cuda()
+    o_dev = h3.packed_mmrope_attention(wl.segments, to_dev(q), to_dev(k), to_dev(v), perm=dperm)
+    hperm = None if perm is None else torch.from_numpy(perm.astype(np.int32))
+    o_host = h3.packed_mmrope_attention_host(wl.segments, _host(q, True), _host(k, True), _host(v, True),
+                                             perm=hperm, heads_per_chunk=0)
+    torch.cuda.current_stream().synchronize()
+    assert h3.h3_check_device_error() == h3.H3_OK
+    assert torch.equal(o_host, o_dev.cpu())
+
+
 def test_host_path_rejects_bad_workspace(h3):
     wl = W.workload(0)
     q, k, v = (_host(a, True) for a in W.qkv_bf16(wl))
