@@ -307,6 +307,22 @@ def test_fused_q_rope_is_identical_to_rotating_first(h3, cfg, layout, rule):
     check_attention(bf16_bits_to_f64(from_dev_bf16(o_fus)), ref, f"fused {wl.name}")
 
 
+@pytest.mark.slow
+def test_fused_q_rope_full_size_ref2va(h3):
+    # the Ref2VA-shaped workload in full (31,952 rows x 42 heads, reference audio
+    # at t down to about -6,000): rotating Q inside the attention kernel from the
+    # (cos, sin) table gives exactly the rotate-first output, in every CTA
+    wl = W.workload(4)
+    perm = W.permutation(wl)
+    q, k, v = W.qkv_bf16(wl)
+    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+    args = dict(perm=_perm_dev(perm), theta=wl.theta, sections=wl.sections)
+    o_sep = h3.packed_mmrope_attention(wl.segments, dq, dk, dv, **args)
+    o_fus = h3.packed_mmrope_attention(wl.segments, dq, dk, dv, fused_q_rope=True, **args)
+    _sync_ok(h3)
+    assert torch.equal(o_sep, o_fus)
+
+
 @pytest.mark.parametrize("cfg,rule", [(0, 0), (4, 0), (1, 1)])
 def test_rope_table_matches_the_oracle_angles(h3, cfg, rule):
     # h3_rope_cos_sin: (cos, sin) of the angle of the fp32 coordinate, each
