@@ -327,7 +327,9 @@ uint64_t h3_host_workspace_bytes(int64_t n_rows, int32_t n_heads);
  *                     is ordered after the last copy out: synchronise `stream`
  *                     to wait for h_o.  Host buffers must stay valid until then.
  * Errors: as the three calls it composes; H3_ERR_INVALID_ARG for a NULL or
- * misaligned workspace; H3_ERR_CUDA if an internal stream or event cannot be
+ * misaligned workspace; H3_ERR_UNSUPPORTED if the chunk plan needs more than
+ * 64 chunks (always when heads_per_chunk < n_heads / 64; with 0 the library's
+ * chunks hold 2 to 8 heads); H3_ERR_CUDA if an internal stream or event cannot be
  * created (they are created once per device and kept until h3_shutdown).
  * Every argument, the segment table included, is checked before anything is
  * queued.  If a CUDA call fails after copies were queued, `stream` is still

@@ -1,8 +1,10 @@
 // h3.cu -- the C ABI of libh3 (declared in include/h3.h).
 //
 // Host-side argument validation, TMA tensor-map encoding and kernel launches.
-// The library allocates no device memory; the per-device error word is a
-// static __device__ variable of this module.
+// The library calls no device allocator: its device memory is static
+// __device__ data of this module (the per-stream error words and the fixed
+// scratch array of the allocation-free host call), and the host-buffer
+// pipeline keeps two streams and a set of events per device.
 #include <algorithm>
 #include <atomic>
 #include <cmath>
@@ -354,7 +356,8 @@ namespace {
 struct HostPipe {
   std::mutex enqueue;             // one caller at a time enqueues on a device
   cudaStream_t h2d = nullptr, d2h = nullptr;
-  static constexpr int kEvents = 3 * 64 + 2;
+  static constexpr int kMaxChunks = 64;
+  static constexpr int kEvents = 2 * kMaxChunks + 2;   // per chunk: copied in, attended; start, end
   cudaEvent_t ev[kEvents] = {};
   bool ok = false;
 };
@@ -370,10 +373,18 @@ HostPipe* host_pipe() {
   std::lock_guard<std::mutex> lock(mu);
   HostPipe& hp = pipes[dev];
   if (!hp.ok) {
-    if (cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
-    if (cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    bool made = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+                cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess;
     for (auto& e : hp.ev)
-      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+      made = made && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+    if (!made) {   // release whatever was created; the next call tries again
+      for (auto& e : hp.ev)
+        if (e != nullptr) cudaEventDestroy(e), e = nullptr;
+      if (hp.h2d != nullptr) cudaStreamDestroy(hp.h2d);
+      if (hp.d2h != nullptr) cudaStreamDestroy(hp.d2h);
+      hp.h2d = hp.d2h = nullptr;
+      return nullptr;
+    }
     hp.ok = true;
   }
   return &hp;
@@ -420,15 +431,15 @@ int pick_heads_per_chunk(int64_t n_rows, int n_heads) {
 // Chunk sizes of the host pipeline: chunks of `hc` heads, and with `taper` the
 // last hc + (n_heads mod hc) heads in halving pieces (6 -> 3, 2, 1), so that the
 // attention and the copy out that remain after the last copy in are short.
-int plan_chunks(int n_heads, int hc, bool taper, int (&sizes)[64]) {
+int plan_chunks(int n_heads, int hc, bool taper, int (&sizes)[HostPipe::kMaxChunks]) {
   int n = 0, left = n_heads;
   const int tail = taper ? std::min(n_heads, hc + n_heads % hc) : 0;
-  while (left > tail && n < 64) {
+  while (left > tail && n < HostPipe::kMaxChunks) {
     const int c = std::min(hc, left - tail);
     sizes[n++] = c;
     left -= c;
   }
-  while (left > 0 && n < 64) {
+  while (left > 0 && n < HostPipe::kMaxChunks) {
     const int c = (left + 1) / 2;
     sizes[n++] = c;
     left -= c;
@@ -455,7 +466,7 @@ h3_status h3_packed_mmrope_attention_host(const h3_segment* segs, int32_t nseg, 
   if (n_rows >= (1ll << 31)) return H3_ERR_INVALID_ARG;
   if (d_work == nullptr || (reinterpret_cast<uintptr_t>(d_work) & 255u)) return H3_ERR_INVALID_ARG;
   const int hc = heads_per_chunk > 0 ? heads_per_chunk : pick_heads_per_chunk(n_rows, n_heads);
-  int chunk_heads[64];
+  int chunk_heads[HostPipe::kMaxChunks];
   const int nchunks = plan_chunks(n_heads, hc, heads_per_chunk == 0, chunk_heads);
   if (nchunks < 0) return H3_ERR_UNSUPPORTED;
   HostPipe* hp = host_pipe();
@@ -473,8 +484,8 @@ h3_status h3_packed_mmrope_attention_host(const h3_segment* segs, int32_t nseg, 
   int32_t* dperm = reinterpret_cast<int32_t*>(w + 4 * t + up(static_cast<uint64_t>(n_rows) * 12u));
 
   cudaEvent_t* ev_in = hp->ev;
-  cudaEvent_t* ev_out = hp->ev + 64;
-  cudaEvent_t ev_start = hp->ev[192], ev_end = hp->ev[193];
+  cudaEvent_t* ev_out = hp->ev + HostPipe::kMaxChunks;
+  cudaEvent_t ev_start = hp->ev[2 * HostPipe::kMaxChunks], ev_end = hp->ev[2 * HostPipe::kMaxChunks + 1];
   auto ck = [](cudaError_t e) { return e == cudaSuccess; };
   // After a failure with copies already queued: order `stream` after both copy
   // streams, so that a caller who synchronises `stream` and then frees its
