@@ -33,11 +33,25 @@ def _stream(stream=None) -> int:
     return int(s.cuda_stream)
 
 
+def _on_device(t, what: str) -> None:
+    """Raise unless ``t`` lives on the current CUDA device (the library dereferences it there)."""
+    import torch
+    if not t.is_cuda or t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{what} must be on the current CUDA device")
+
+
+def _exact(t, dtype, shape, what: str) -> None:
+    """Raise unless ``t`` is a contiguous tensor of exactly this dtype and shape."""
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{what} must be a contiguous {dtype} tensor of shape {tuple(shape)}")
+
+
 def _row_layout(x):
     """(batch, n_rows, n_heads, row_stride) of a [.., N, H, 128] bf16 view."""
     import torch
     if x.dtype != torch.bfloat16 or not x.is_cuda:
         raise TypeError("expected a CUDA bf16 tensor")
+    _on_device(x, "Q, K, V and O")
     if x.dim() not in (3, 4) or x.shape[-1] != 128 or x.stride(-1) != 1 or x.stride(-2) != 128:
         raise ValueError("expected [N, H, 128] or [B, N, H, 128] with heads contiguous")
     n, h = x.shape[-3], x.shape[-2]
@@ -53,10 +67,13 @@ def build_coords(segments, n_rows: int, perm=None, out=None, stream=None):
     import torch
     if out is None:
         out = torch.empty((n_rows, 3), dtype=torch.float32, device="cuda")
+    _exact(out, torch.float32, (n_rows, 3), "out")
+    _on_device(out, "out")
     p = 0
     if perm is not None:
-        if perm.dtype != torch.int32 or not perm.is_cuda or perm.numel() != n_rows:
-            raise ValueError("perm must be a CUDA int32 tensor of n_rows entries")
+        if perm.dtype != torch.int32 or not perm.is_cuda or perm.numel() != n_rows or not perm.is_contiguous():
+            raise ValueError("perm must be a contiguous CUDA int32 tensor of n_rows entries")
+        _on_device(perm, "perm")
         p = perm.data_ptr()
     h3_build_coords(segments, p, n_rows, out.data_ptr(), _stream(stream))
     return out
@@ -81,6 +98,7 @@ def mmrope_qk(q, k, coords, q_out=None, k_out=None, theta=10000.0, sections=(32,
         raise ValueError("outputs must share the inputs' layout")
     if coords.dtype != torch.float32 or coords.numel() != 3 * b * n or not coords.is_contiguous():
         raise ValueError("coords must be contiguous fp32 [rows, 3]")
+    _on_device(coords, "coords")
     h3_mmrope_qk(q.data_ptr() if q is not None else 0, k.data_ptr(),
                  q_out.data_ptr() if q is not None else 0, k_out.data_ptr(), coords.data_ptr(), b * n, h,
                  rs, rope_cfg(theta, 128, sections, pair_layout, freq_rule), _stream(stream))
@@ -93,11 +111,13 @@ def rope_cos_sin(coords, out=None, theta=10000.0, sections=(32, 48, 48), pair_la
     import torch
     if coords.dtype != torch.float32 or coords.dim() != 2 or coords.shape[1] != 3 or not coords.is_contiguous():
         raise ValueError("coords must be contiguous fp32 [rows, 3]")
+    _on_device(coords, "coords")
     n = coords.shape[0]
     if out is None:
         out = torch.empty((n, 64, 2), dtype=torch.float32, device=coords.device)
     if out.dtype != torch.float32 or out.numel() != n * 128 or not out.is_contiguous():
         raise ValueError("out must be contiguous fp32 [rows, 64, 2]")
+    _on_device(out, "out")
     h3_rope_cos_sin(coords.data_ptr(), n, rope_cfg(theta, 128, sections, pair_layout, freq_rule), out.data_ptr(),
                     _stream(stream))
     return out
@@ -123,11 +143,13 @@ def packed_attention(q, k, v, out=None, lse=None, softmax_scale: float = 0.0, st
     if lse is not None:
         if lse.dtype != torch.float32 or lse.numel() != b * h * n or not lse.is_contiguous():
             raise ValueError("lse must be contiguous fp32 [B, H, N]")
+        _on_device(lse, "lse")
         lp = lse.data_ptr()
     cp, cfg = 0, None
     if rope_cs is not None:
         if rope_cs.dtype != torch.float32 or rope_cs.numel() != 128 * b * n or not rope_cs.is_contiguous():
             raise ValueError("rope_cs must be contiguous fp32 [rows, 64, 2]")
+        _on_device(rope_cs, "rope_cs")
         cp, cfg = rope_cs.data_ptr(), rope_cfg(theta, 128, sections, pair_layout, freq_rule)
     h3_packed_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lp, b, n, h, rs,
                         softmax_scale, d_rope_cs=cp, cfg=cfg, stream=_stream(stream))
@@ -177,18 +199,26 @@ def packed_mmrope_attention_host(segments, q, k, v, out=None, perm=None, workspa
     Work is queued on ``stream``; synchronise it before reading the output.
     """
     import torch
+    if q.dim() != 3 or q.shape[-1] != 128:
+        raise ValueError("expected [N, H, 128]")
     for t in (q, k, v):
         if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != q.shape:
             raise ValueError("q, k, v must be contiguous CPU bf16 tensors of one shape")
-    n, h = q.shape[-3], q.shape[-2]
-    if q.dim() != 3 or q.shape[-1] != 128:
-        raise ValueError("expected [N, H, 128]")
+    n, h = q.shape[0], q.shape[1]
     if out is None:
         out = torch.empty_like(q, pin_memory=q.is_pinned())
-    if perm is not None and (perm.dtype != torch.int32 or perm.is_cuda or perm.numel() != n):
-        raise ValueError("perm must be a CPU int32 tensor of N entries")
+    if out.is_cuda:
+        raise ValueError("out must be a CPU tensor")
+    _exact(out, torch.bfloat16, q.shape, "out")
+    if perm is not None and (perm.dtype != torch.int32 or perm.is_cuda or perm.numel() != n
+                             or not perm.is_contiguous()):
+        raise ValueError("perm must be a contiguous CPU int32 tensor of N entries")
     if workspace is None:
         workspace = host_workspace(n, h)
+    need = h3_host_workspace_bytes(n, h)
+    if workspace.dtype != torch.uint8 or not workspace.is_contiguous() or workspace.numel() < need:
+        raise ValueError(f"workspace must be a contiguous uint8 tensor of at least {need} bytes")
+    _on_device(workspace, "workspace")
     h3_packed_mmrope_attention_host(segments, perm.data_ptr() if perm is not None else 0, q.data_ptr(),
                                     k.data_ptr(), v.data_ptr(), out.data_ptr(), workspace.data_ptr(), n, h,
                                     rope_cfg(theta, 128, sections, pair_layout, freq_rule), heads_per_chunk,
@@ -207,12 +237,18 @@ def adaln_modulate(x, timestep_index, token_tag, table, out=None, eps: float = 1
         raise ValueError("x must be a CUDA bf16 [N, C] tensor with unit inner stride")
     n, c = x.shape
     out = torch.empty_like(x) if out is None else out
+    if out.dtype != torch.bfloat16 or tuple(out.shape) != (n, c) or out.stride(1) != 1:
+        raise ValueError("out must be a bf16 [N, C] tensor with unit inner stride")
+    for t, what in ((x, "x"), (out, "out")):
+        _on_device(t, what)
     for t in (timestep_index, token_tag):
         if t.dtype != torch.int32 or t.numel() != n or not t.is_contiguous() or not t.is_cuda:
             raise ValueError("indices must be contiguous CUDA int32 [N]")
+        _on_device(t, "indices")
     if table.dtype != torch.float32 or table.dim() != 3 or tuple(table.shape[1:]) != (2, c) \
             or not table.is_contiguous():
         raise ValueError("table must be contiguous fp32 [E, 2, C]")
+    _on_device(table, "table")
     h3_adaln_modulate(x.data_ptr(), out.data_ptr(), timestep_index.data_ptr(), token_tag.data_ptr(),
                       table.data_ptr(), table.shape[0], n, c, x.stride(0), out.stride(0), eps, _stream(stream))
     return out

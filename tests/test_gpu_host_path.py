@@ -65,8 +65,9 @@ def test_host_path_tapered_chunks_many_heads(h3, heads):
 def test_host_path_rejects_bad_workspace(h3):
     wl = W.workload(0)
     q, k, v = (_host(a, True) for a in W.qkv_bf16(wl))
-    ws = h3.host_workspace(wl.n_rows, wl.heads)
+    need = h3.h3_host_workspace_bytes(wl.n_rows, wl.heads)
+    ws = torch.empty(need + 256, dtype=torch.uint8, device="cuda")
     with pytest.raises(h3.H3Error) as e:
         h3.packed_mmrope_attention_host(wl.segments, q, k, v, perm=torch.zeros(82, dtype=torch.int32),
-                                        workspace=ws[8:])      # misaligned
+                                        workspace=ws[8:8 + need])      # large enough, misaligned
     assert e.value.status == h3.H3_ERR_INVALID_ARG
