@@ -15,6 +15,8 @@ What it computes (plain definitions, fp64 unless stated):
                    head over all packed rows (non-causal, no mask).
 * ``clock``     -- the time-unit facts the pages state (40 Hz audio ticks,
                    5/3 ticks per 24 fps source frame, 4x temporal stride).
+* ``adaln``     -- per-row AdaLN modulation: LayerNorm without its own affine,
+                   then (1 + scale[e]) and shift[e] with e = timestep * 3 + tag.
 
 Sources (page titles as published):
   [P1] "Inside MiniMax H3: One DiT Stream for Text, Video, and Stereo Audio"
@@ -30,5 +32,5 @@ Sources (page titles as published):
 Every function is pinned by a ``-m "not gpu"`` test against facts the pages
 print or against closed forms and invariants; none is "parity unpinned".
 """
-from . import clock, coords, rope, attention  # noqa: F401
+from . import adaln, clock, coords, rope, attention  # noqa: F401
 from .pipeline import packed_mmrope_attention, rotated_qk  # noqa: F401
